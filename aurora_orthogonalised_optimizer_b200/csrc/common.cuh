@@ -1,0 +1,111 @@
+// Shared device-side helpers of libaurora_muon: dtype access, reductions,
+// the sticky status word and the per-launch matrix tables.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/aurora_muon.h"
+
+namespace am {
+
+constexpr int kF32 = MUON_F32;
+constexpr int kBF16 = MUON_BF16;
+
+// ---------------------------------------------------------------- dtype access
+__device__ __forceinline__ float ld_as_f32(const void* p, int64_t i, int dt) {
+  if (dt == kBF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return reinterpret_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void st_from_f32(void* p, int64_t i, int dt, float v) {
+  if (dt == kBF16) reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(p)[i] = v;
+}
+__host__ __device__ __forceinline__ int dt_bytes(int dt) { return dt == kBF16 ? 2 : 4; }
+
+// ---------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Deterministic block sum of one double per thread (blockDim.x multiple of 32,
+// at most 1024).  Every thread gets the result.
+__device__ __forceinline__ double block_sum(double v, double* smem32) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) smem32[wid] = v;
+  __syncthreads();
+  double t = 0.0;
+  for (int w = 0; w < nw; ++w) t += smem32[w];
+  return t;
+}
+
+// ---------------------------------------------------------------- tables
+// Matrix descriptor for the element-wise / reduction kernels.  Original
+// orientation is m x n; the "X orientation" is s x l (s = min, l = max), the
+// transpose of the original when the matrix is tall (m > n).
+struct MatDesc {
+  void* W;            // param (param dtype), original orientation
+  const void* G;      // grad / input (grad dtype), original orientation
+  float* M;           // momentum fp32, original orientation
+  float* V;           // optional fp32 output, original orientation
+  void* uX;           // u in X orientation (ns dtype), leading dim ldl
+  void* UX;           // polar output in X orientation (ns dtype), leading dim ldl
+  void* X0;           // scaled Newton-Schulz input (ns dtype), leading dim ldl
+  float* D;           // Aurora column scale (length l)
+  float* vec0;        // power-iteration vectors (length >= l), two of them
+  float* vec1;
+  float* rho_slot;    // bucket-ordered copy of rho read by the GEMM epilogues
+  int64_t m, n, s, l, ldl;
+  int tall;           // m > n
+  int idx;            // matrix index (scalar block row)
+  int part;           // first partial slot of this matrix
+  int nblk;           // blocks of this matrix in the current launch
+  int flag;           // launch-specific per-matrix flag
+};
+
+constexpr int kMaxMatsPerLaunch = 96;
+
+struct MatTable {
+  int count;
+  int ns_dtype;       // dtype of uX / UX / X0
+  int param_dtype;
+  int grad_dtype;
+  int blk_prefix[kMaxMatsPerLaunch + 1];
+  MatDesc mats[kMaxMatsPerLaunch];
+};
+
+__device__ __forceinline__ int find_mat(const MatTable& t, int blk) {
+  int lo = 0, hi = t.count - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (t.blk_prefix[mid] <= blk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Per-matrix scalar block (doubles), indexed by MatDesc::idx.
+enum ScalarSlot {
+  S_SUM_U2 = 0,    // |u|_F^2
+  S_SUM_W2,        // |W|_F^2
+  S_SUM_X02,       // |X0|_F^2 of the scaled NS input
+  S_RHO,           // 1 / (|X0|_F + ns_eps)
+  S_SIGMA,         // operator-norm estimate
+  S_SUM_UU2,       // |U|_F^2 of the polar output
+  S_DOT_UUX,       // <U, u>
+  S_COEF_U,        // final coefficient of U in V
+  S_COEF_u,        // final coefficient of u in V
+  S_VNORM2,        // scratch
+  S_COUNT = 16
+};
+
+}  // namespace am

@@ -1,0 +1,763 @@
+// Host engine of libaurora_muon: argument validation, shape bucketing,
+// workspace carving, the stage sequence of one optimizer step, and the C ABI
+// declared in include/aurora_muon.h.
+//
+// Stage order of muon_step (Track 3 write-up, "组合优化栈" + "u/w-floor"):
+//   prologue (momentum, Nesterov, u in X orientation, |u|^2, |W|^2)
+//   [contra]  power iteration on u -> sigma
+//   [aurora]  D init from the tall-oriented row norms of u
+//   polar loop: scaled input X0 -> rho; ns_steps x {Gram, square, update}
+//               [aurora, not last] D update from the row norms of U
+//   <U,U>, <U,u> -> per-matrix coefficients -> fused epilogue W <- W - lr V
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "kernels.h"
+
+using namespace am;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
+
+struct MatPlan {
+  int64_t m, n, s, l;
+  int tall, bucket, bidx;
+  int64_t part;      // first partial block slot
+};
+
+struct BucketPlan {
+  int64_t s, l, ldl, lds;
+  std::vector<int> members;
+  size_t off_uX, off_P, off_Q, off_A, off_B, off_D, off_v0, off_v1, off_rho;
+};
+
+struct Plan {
+  int ns_dtype = kBF16;
+  int nsb = 2;
+  std::vector<MatPlan> mats;
+  std::vector<BucketPlan> buckets;
+  size_t off_scal = 0, off_partials = 0, total = 0;
+};
+
+int ns_dtype_of(const muon_config* c) { return c->gemm_mode == MUON_GEMM_FP32 ? kF32 : kBF16; }
+
+Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
+  Plan p;
+  p.ns_dtype = ns_dtype_of(cfg);
+  p.nsb = dt_bytes(p.ns_dtype);
+  std::map<std::pair<int64_t, int64_t>, int> bmap;
+  int64_t part = 0;
+  for (int i = 0; i < n; ++i) {
+    MatPlan mp;
+    mp.m = shapes[i].rows;
+    mp.n = shapes[i].cols;
+    mp.s = std::min(mp.m, mp.n);
+    mp.l = std::max(mp.m, mp.n);
+    mp.tall = mp.m > mp.n;
+    auto key = std::make_pair(mp.s, mp.l);
+    auto it = bmap.find(key);
+    if (it == bmap.end()) {
+      BucketPlan b{};
+      b.s = mp.s;
+      b.l = mp.l;
+      b.ldl = round8(mp.l);
+      b.lds = round8(mp.s);
+      p.buckets.push_back(b);
+      it = bmap.emplace(key, (int)p.buckets.size() - 1).first;
+    }
+    mp.bucket = it->second;
+    mp.bidx = (int)p.buckets[mp.bucket].members.size();
+    p.buckets[mp.bucket].members.push_back(i);
+    mp.part = part;
+    const int64_t tiles = cdiv(mp.m, 64) * cdiv(mp.n, 64);
+    part += std::max(tiles, cdiv(mp.m * mp.n, 4096));
+    p.mats.push_back(mp);
+  }
+  size_t off = 0;
+  for (auto& b : p.buckets) {
+    const size_t cnt = b.members.size();
+    const size_t xbytes = cnt * (size_t)b.s * (size_t)b.ldl * p.nsb;
+    const size_t abytes = cnt * (size_t)b.s * (size_t)b.lds * p.nsb;
+    b.off_uX = off; off = align_up(off + xbytes);
+    b.off_P = off;  off = align_up(off + xbytes);
+    b.off_Q = off;  off = align_up(off + xbytes);
+    b.off_A = off;  off = align_up(off + abytes);
+    b.off_B = off;  off = align_up(off + abytes);
+    b.off_D = off;  off = align_up(off + cnt * (size_t)b.l * 4);
+    b.off_v0 = off; off = align_up(off + cnt * (size_t)b.l * 4);
+    b.off_v1 = off; off = align_up(off + cnt * (size_t)b.l * 4);
+    b.off_rho = off; off = align_up(off + cnt * 4);
+  }
+  p.off_scal = off;
+  off = align_up(off + (size_t)n * S_COUNT * sizeof(double));
+  p.off_partials = off;
+  off = align_up(off + (size_t)part * 2 * sizeof(double));
+  p.total = off;
+  return p;
+}
+
+// ---------------------------------------------------------------- validation
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+muon_status check_config(const muon_config* c, bool need_ns, bool need_pp, bool need_pi) {
+  if (!c) return MUON_ERR_INVALID_ARG;
+  if (c->gemm_mode < 0 || c->gemm_mode > 2) return MUON_ERR_INVALID_ARG;
+  if (c->param_dtype < 0 || c->param_dtype > 1 || c->grad_dtype < 0 || c->grad_dtype > 1)
+    return MUON_ERR_INVALID_ARG;
+  if (need_ns && c->ns_steps < 1) return MUON_ERR_INVALID_ARG;
+  if (need_pp && c->pp_iterations < 1) return MUON_ERR_INVALID_ARG;
+  if (need_pi && c->power_iters < 1) return MUON_ERR_INVALID_ARG;
+  if (c->weight_decay != 0.f) return MUON_ERR_INVALID_ARG;
+  if (!(c->ns_eps >= 0.f) || !(c->pp_eps > 0.f) || !(c->target_uw >= 0.f)) return MUON_ERR_INVALID_ARG;
+  return MUON_OK;
+}
+
+muon_status check_shapes(int n, const muon_shape* shapes) {
+  if (n < 0) return MUON_ERR_INVALID_ARG;
+  if (n > 0 && !shapes) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (shapes[i].rows <= 0 || shapes[i].cols <= 0) return MUON_ERR_INVALID_ARG;
+    if (shapes[i].rows > (int64_t)1 << 31 || shapes[i].cols > (int64_t)1 << 31) return MUON_ERR_INVALID_ARG;
+    if (std::min(shapes[i].rows, shapes[i].cols) > 32768) return MUON_ERR_UNSUPPORTED;
+  }
+  return MUON_OK;
+}
+
+template <class P>
+muon_status check_ptrs(int n, P const* arr, bool allow_null_array, bool allow_null_entry) {
+  if (n == 0) return MUON_OK;
+  if (!arr) return allow_null_array ? MUON_OK : MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!arr[i]) { if (allow_null_entry) continue; return MUON_ERR_INVALID_ARG; }
+    if (!aligned16((const void*)arr[i])) return MUON_ERR_INVALID_ARG;
+  }
+  return MUON_OK;
+}
+
+muon_status check_ws(const Plan& p, void* ws, size_t bytes) {
+  if (p.total == 0) return MUON_OK;
+  if (!ws || bytes < p.total || !aligned16(ws)) return MUON_ERR_WORKSPACE;
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- device info
+int num_sms_current() {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> g(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cache[dev] = sms;
+  return sms;
+}
+
+// ---------------------------------------------------------------- tracing
+enum ProfClass { PC_GEMM_TC = 0, PC_GEMM_SIMT, PC_PROLOGUE, PC_POWER, PC_AURORA, PC_REDUCE, PC_EPILOGUE, PC_COUNT };
+const char* const kProfNames[PC_COUNT] = {"ns_gemm_tc", "ns_gemm_simt", "prologue", "power_iter",
+                                          "aurora_rows", "reductions", "epilogue"};
+
+struct ProfRecord {
+  int cls;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+
+struct ProfState {
+  std::mutex mu;
+  bool on = false;
+  std::vector<ProfRecord> recs;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pool;
+  size_t used = 0;
+} g_prof;
+
+// Brackets one launch with events when tracing is on.
+struct ProfScope {
+  ProfRecord rec{};
+  bool active = false;
+  cudaStream_t st;
+  ProfScope(int cls, double flops, double bytes, cudaStream_t s) : st(s) {
+    std::lock_guard<std::mutex> g(g_prof.mu);
+    if (!g_prof.on) return;
+    if (g_prof.used == g_prof.pool.size()) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess) return;
+      if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return; }
+      g_prof.pool.emplace_back(a, b);
+    }
+    auto ev = g_prof.pool[g_prof.used++];
+    rec = ProfRecord{cls, ev.first, ev.second, flops, bytes};
+    active = cudaEventRecord(rec.a, st) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!active) return;
+    cudaEventRecord(rec.b, st);
+    std::lock_guard<std::mutex> g(g_prof.mu);
+    g_prof.recs.push_back(rec);
+  }
+};
+
+// ---------------------------------------------------------------- context
+struct Ctx {
+  const muon_config* cfg;
+  const Plan* plan;
+  char* ws;
+  cudaStream_t st;
+  double* scal;
+  double* partials;
+  void* const* W;
+  const void* const* G;
+  float* const* M;
+  float* const* V;
+  int param_dtype, grad_dtype;
+};
+
+template <class T> T* wsp(const Ctx& c, size_t off) { return reinterpret_cast<T*>(c.ws + off); }
+
+MatDesc make_desc(const Ctx& c, int i) {
+  const MatPlan& mp = c.plan->mats[i];
+  const BucketPlan& b = c.plan->buckets[mp.bucket];
+  const int nsb = c.plan->nsb;
+  const size_t xo = (size_t)mp.bidx * b.s * b.ldl * nsb;
+  MatDesc d{};
+  d.W = c.W ? c.W[i] : nullptr;
+  d.G = c.G ? c.G[i] : nullptr;
+  d.M = c.M ? c.M[i] : nullptr;
+  d.V = c.V ? c.V[i] : nullptr;
+  d.uX = c.ws + b.off_uX + xo;
+  const bool odd = (c.cfg->ns_steps & 1) != 0;
+  d.UX = c.ws + (odd ? b.off_P : b.off_Q) + xo;
+  d.X0 = c.ws + b.off_Q + xo;
+  d.D = wsp<float>(c, b.off_D) + (size_t)mp.bidx * b.l;
+  d.vec0 = wsp<float>(c, b.off_v0) + (size_t)mp.bidx * b.l;
+  d.vec1 = wsp<float>(c, b.off_v1) + (size_t)mp.bidx * b.l;
+  d.rho_slot = wsp<float>(c, b.off_rho) + mp.bidx;
+  d.m = mp.m; d.n = mp.n; d.s = mp.s; d.l = mp.l; d.ldl = b.ldl;
+  d.tall = mp.tall;
+  d.idx = i;
+  d.part = (int)mp.part;
+  return d;
+}
+
+// Run `launch(table, nblk_total)` over `ids` in chunks of at most
+// kMaxMatsPerLaunch matrices; blocks(d) gives each matrix's block count and
+// may set d.flag.
+template <class BlocksFn, class LaunchFn>
+cudaError_t for_chunks(const Ctx& c, const std::vector<int>& ids, BlocksFn blocks, LaunchFn launch) {
+  size_t k = 0;
+  while (k < ids.size()) {
+    MatTable t;
+    std::memset(&t, 0, sizeof(t));
+    t.ns_dtype = c.plan->ns_dtype;
+    t.param_dtype = c.param_dtype;
+    t.grad_dtype = c.grad_dtype;
+    int total = 0;
+    while (k < ids.size() && t.count < kMaxMatsPerLaunch) {
+      MatDesc d = make_desc(c, ids[k]);
+      d.nblk = (int)blocks(d);
+      t.blk_prefix[t.count] = total;
+      total += d.nblk;
+      t.mats[t.count++] = d;
+      ++k;
+    }
+    t.blk_prefix[t.count] = total;
+    cudaError_t e = launch(t, total);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+double table_elems(const MatTable& t) {
+  double e = 0;
+  for (int i = 0; i < t.count; ++i) e += (double)t.mats[i].m * (double)t.mats[i].n;
+  return e;
+}
+
+int64_t tiles_orig(const MatDesc& d) { return cdiv(d.m, 64) * cdiv(d.n, 64); }
+int64_t tiles_x(const MatDesc& d) { return cdiv(d.s, 64) * cdiv(d.l, 64); }
+
+#define CK(expr)                                   \
+  do {                                             \
+    cudaError_t _e = (expr);                       \
+    if (_e != cudaSuccess) return MUON_ERR_CUDA;   \
+  } while (0)
+
+// ---------------------------------------------------------------- stages
+muon_status stage_prologue(const Ctx& c, const std::vector<int>& ids, int mode, bool want_w2) {
+  const double per_elem = dt_bytes(c.grad_dtype) + c.plan->nsb + (mode == 0 ? 8.0 : 0.0) +
+                          (want_w2 ? dt_bytes(c.param_dtype) : 0.0);
+  CK(for_chunks(c, ids, tiles_orig, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
+    return launch_prologue(t, nb, mode, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
+  }));
+  CK(for_chunks(c, ids, tiles_orig, [&](const MatTable& t, int) {
+    ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
+    return launch_finalize_sums(t, c.partials, 2, S_SUM_U2, want_w2 ? S_SUM_W2 : -1, c.scal, c.st);
+  }));
+  return MUON_OK;
+}
+
+// Power iteration on u (X orientation): sigma in S_SIGMA.
+// With A the stored matrix and v over A's columns: t = A v, w = A^T t.
+// Wide/square (X = A): t is a row dot of X, w a column dot.
+// Tall (X = A^T):      t is a column dot of X, w a row dot.
+// k_matvec flag: 0 = row dot (in: l, out: s), 1 = column dot (in: s, out: l).
+muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int iters) {
+  auto vec_blocks = [](MatDesc& d) -> int64_t { d.flag = d.tall ? 1 : 0; return 0; };
+  auto vecop = [&](int which, int mode, int len_is_s_when_flag0) {
+    return for_chunks(c, ids, vec_blocks, [&](const MatTable& t, int) {
+      ProfScope ps(PC_POWER, 0.0, 0.0, c.st);
+      return launch_vecop(t, which, mode, len_is_s_when_flag0, c.scal, c.st);
+    });
+  };
+  auto pass = [&](bool first, int dir) {
+    return for_chunks(c, ids, [first](MatDesc& d) -> int64_t {
+      const bool rowdot = first ? !d.tall : (bool)d.tall;
+      d.flag = rowdot ? 0 : 1;
+      return rowdot ? cdiv(d.s, 8) : cdiv(d.l, 64);
+    }, [&](const MatTable& t, int nb) {
+      ProfScope ps(PC_POWER, 2.0 * table_elems(t), c.plan->nsb * table_elems(t), c.st);
+      return launch_matvec(t, nb, dir, c.st);
+    });
+  };
+  CK(vecop(0, 0, 0));          // v = ones / sqrt(len(v)) on vec0
+  for (int k = 0; k < iters; ++k) {
+    CK(pass(true, 0));         // t = A v    (vec0 -> vec1)
+    CK(pass(false, 1));        // w = A^T t  (vec1 -> vec0)
+    CK(vecop(0, 1, 0));        // v = w / |w|
+  }
+  CK(pass(true, 0));           // t = A v
+  CK(vecop(1, 2, 1));          // sigma = |t|
+  return MUON_OK;
+}
+
+// Algorithmic flops of a launch: 2 K per useful output element; the
+// symmetric kinds need only the s (s + 1) / 2 elements of one triangle.
+double gemm_flops(const GemmLaunch& L) {
+  double f = 0;
+  for (int g = 0; g < L.num_groups; ++g) {
+    const GemmGroup& G = L.g[g];
+    const double outs = (G.kind == GK_UPD) ? (double)G.M * G.N : 0.5 * (double)G.M * (G.M + 1);
+    f += 2.0 * G.K * outs * G.count;
+  }
+  return f;
+}
+
+muon_status gemm_launch(const Ctx& c, GemmLaunch& L) {
+  if (L.num_groups == 0) return MUON_OK;
+  if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
+    alignas(64) unsigned char maps[kMaxGemmGroups * 2 * 128];
+    if (!tc_encode_maps(L, maps)) return MUON_ERR_CUDA;
+    ProfScope ps(PC_GEMM_TC, gemm_flops(L), 0.0, c.st);
+    CK(launch_gemm_tc(L, maps, num_sms_current(), c.st));
+  } else {
+    ProfScope ps(PC_GEMM_SIMT, gemm_flops(L), 0.0, c.st);
+    CK(launch_gemm_simt(L, c.st));
+  }
+  L.num_groups = 0;
+  L.total_tiles = 0;
+  return MUON_OK;
+}
+
+void add_group(const Ctx& c, GemmLaunch& L, GemmGroup g) {
+  if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
+    g.tiles_per_mat = tc_tile_count(g.kind, g.M, g.N, &g.tiles_m, &g.tiles_n);
+  } else {
+    g.tiles_m = (int)cdiv(g.M, 64);
+    g.tiles_n = (int)cdiv(g.N, 64);
+    g.tiles_per_mat = g.tiles_m * g.tiles_n;
+  }
+  g.tile_begin = L.total_tiles;
+  L.g[L.num_groups++] = g;
+  L.total_tiles += g.tiles_per_mat * g.count;
+}
+
+// ns_steps Newton-Schulz iterations on every matrix of the given buckets.
+// it = 0 reads X0 (uX, or Q when x0_in_Q) scaled by rho; output ping-pongs
+// P (even it), Q (odd it).
+muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids, bool x0_in_Q) {
+  const Plan& p = *c.plan;
+  const float a = c.cfg->ns_a, bc = c.cfg->ns_b, cc = c.cfg->ns_c;
+  for (int it = 0; it < c.cfg->ns_steps; ++it) {
+    for (int kind = 0; kind < 3; ++kind) {
+      GemmLaunch L;
+      std::memset(&L, 0, sizeof(L));
+      L.dtype = p.ns_dtype;
+      for (int bi : bucket_ids) {
+        const BucketPlan& b = p.buckets[bi];
+        char* X_in = c.ws + (it == 0 ? (x0_in_Q ? b.off_Q : b.off_uX) : ((it & 1) ? b.off_P : b.off_Q));
+        char* X_out = c.ws + ((it & 1) ? b.off_Q : b.off_P);
+        char* Ab = c.ws + b.off_A;
+        char* Bb = c.ws + b.off_B;
+        const int64_t sx = b.s * b.ldl, ss = b.s * b.lds;
+        GemmGroup g{};
+        g.kind = kind;
+        g.count = (int)b.members.size();
+        g.rho = wsp<float>(c, b.off_rho);
+        if (kind == GK_GRAM) {
+          g.M = (int)b.s; g.N = (int)b.s; g.K = (int)b.l;
+          g.A = X_in; g.lda = b.ldl; g.sa = sx;
+          g.B = X_in; g.ldb = b.ldl; g.sb = sx;
+          g.C = Ab; g.ldc = b.lds; g.sc = ss;
+          g.alpha0 = 1.f; g.pa = it == 0 ? 2 : 0;
+        } else if (kind == GK_SQR) {
+          g.M = (int)b.s; g.N = (int)b.s; g.K = (int)b.s;
+          g.A = Ab; g.lda = b.lds; g.sa = ss;
+          g.B = Ab; g.ldb = b.lds; g.sb = ss;
+          g.C = Bb; g.ldc = b.lds; g.sc = ss;
+          g.E = Ab; g.lde = b.lds; g.se = ss;
+          g.alpha0 = cc; g.beta0 = bc;
+          g.rho = nullptr;
+        } else {
+          g.M = (int)b.s; g.N = (int)b.l; g.K = (int)b.s;
+          g.A = Bb; g.lda = b.lds; g.sa = ss;
+          g.B = X_in; g.ldb = b.ldl; g.sb = sx;
+          g.C = X_out; g.ldc = b.ldl; g.sc = sx;
+          g.E = X_in; g.lde = b.ldl; g.se = sx;
+          g.alpha0 = 1.f; g.beta0 = a;
+          g.pa = g.pb = it == 0 ? 1 : 0;
+        }
+        add_group(c, L, g);
+        if (L.num_groups == kMaxGemmGroups) {
+          muon_status s = gemm_launch(c, L);
+          if (s != MUON_OK) return s;
+        }
+      }
+      muon_status s = gemm_launch(c, L);
+      if (s != MUON_OK) return s;
+    }
+  }
+  return MUON_OK;
+}
+
+std::vector<int> ids_of_buckets(const Plan& p, const std::vector<int>& bids) {
+  std::vector<int> ids;
+  for (int b : bids) for (int i : p.buckets[b].members) ids.push_back(i);
+  return ids;
+}
+
+// Polar factor of u (in X orientation) for every matrix; result in UX.
+muon_status stage_polar(const Ctx& c, bool aurora) {
+  const Plan& p = *c.plan;
+  std::vector<int> all_b, sq_b, ns_b;
+  for (int b = 0; b < (int)p.buckets.size(); ++b) {
+    all_b.push_back(b);
+    (p.buckets[b].s == p.buckets[b].l ? sq_b : ns_b).push_back(b);
+  }
+  const std::vector<int> plain_b = aurora ? sq_b : all_b;
+  const float eps = c.cfg->ns_eps;
+  if (!plain_b.empty()) {
+    std::vector<int> ids = ids_of_buckets(p, plain_b);
+    CK(for_chunks(c, ids, [](const MatDesc&) { return (int64_t)0; }, [&](const MatTable& t, int) {
+      ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
+      cudaError_t e = launch_scalars(t, 0, S_SUM_U2, eps, 0.f, 0.f, c.scal, c.st);
+      if (e != cudaSuccess) return e;
+      return launch_copy_rho(t, c.scal, c.st);
+    }));
+    muon_status s = stage_newton_schulz(c, plain_b, false);
+    if (s != MUON_OK) return s;
+  }
+  if (aurora && !ns_b.empty()) {
+    std::vector<int> ids = ids_of_buckets(p, ns_b);
+    const float pe = c.cfg->pp_eps, beta = c.cfg->pp_beta;
+    CK(for_chunks(c, ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
+      ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
+      return launch_colnorm(t, nb, 0, pe, beta, c.st);
+    }));
+    for (int k = 0; k < c.cfg->pp_iterations; ++k) {
+      CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int nb) {
+        ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
+        return launch_scale_cols(t, nb, c.partials, c.st);
+      }));
+      CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int) {
+        ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
+        cudaError_t e = launch_finalize_sums(t, c.partials, 1, S_SUM_X02, -1, c.scal, c.st);
+        if (e != cudaSuccess) return e;
+        e = launch_scalars(t, 0, S_SUM_X02, eps, 0.f, 0.f, c.scal, c.st);
+        if (e != cudaSuccess) return e;
+        return launch_copy_rho(t, c.scal, c.st);
+      }));
+      muon_status s = stage_newton_schulz(c, ns_b, true);
+      if (s != MUON_OK) return s;
+      if (k < c.cfg->pp_iterations - 1)
+        CK(for_chunks(c, ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
+          ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
+          return launch_colnorm(t, nb, 1, pe, beta, c.st);
+        }));
+    }
+  }
+  return MUON_OK;
+}
+
+std::vector<int> iota_ids(int n) {
+  std::vector<int> v(n);
+  for (int i = 0; i < n; ++i) v[i] = i;
+  return v;
+}
+
+// Write V = cU U + cu u (original orientation) and optionally W.
+muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool update_w, float lr) {
+  const bool need_u = c.cfg->contra != 0.f || !update_w;
+  const double per_elem = c.plan->nsb * (need_u ? 2.0 : 1.0) + (update_w ? 2.0 * dt_bytes(c.param_dtype) : 0.0) +
+                          (c.V ? 4.0 : 0.0);
+  CK(for_chunks(c, ids, tiles_orig, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
+    return launch_epilogue(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
+  }));
+  return MUON_OK;
+}
+
+muon_status stage_dots(const Ctx& c, const std::vector<int>& ids) {
+  CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_REDUCE, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
+    return launch_dots(t, nb, c.partials, c.st);
+  }));
+  CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int) {
+    ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
+    return launch_finalize_sums(t, c.partials, 2, S_SUM_UU2, S_DOT_UUX, c.scal, c.st);
+  }));
+  return MUON_OK;
+}
+
+muon_status set_coeffs(const Ctx& c, const std::vector<int>& ids, int op) {
+  CK(for_chunks(c, ids, [](const MatDesc&) { return (int64_t)0; }, [&](const MatTable& t, int) {
+    ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
+    return launch_scalars(t, op, 0, c.cfg->ns_eps, c.cfg->contra, c.cfg->target_uw, c.scal, c.st);
+  }));
+  return MUON_OK;
+}
+
+Ctx make_ctx(const muon_config* cfg, const Plan& p, void* ws, void* stream) {
+  Ctx c{};
+  c.cfg = cfg;
+  c.plan = &p;
+  c.ws = reinterpret_cast<char*>(ws);
+  c.st = reinterpret_cast<cudaStream_t>(stream);
+  c.scal = reinterpret_cast<double*>(c.ws + p.off_scal);
+  c.partials = reinterpret_cast<double*>(c.ws + p.off_partials);
+  c.param_dtype = cfg->param_dtype;
+  c.grad_dtype = cfg->grad_dtype;
+  return c;
+}
+
+// Shared front half of ns_polar / aurora_polar / opnorm_normalize.
+muon_status stage_input(Ctx& c, int n, const void* const* in, int in_dtype) {
+  c.G = in;
+  c.grad_dtype = in_dtype;
+  return stage_prologue(c, iota_ids(n), 1, false);
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+void muon_config_default(muon_config* c) {
+  if (!c) return;
+  std::memset(c, 0, sizeof(*c));
+  c->lr = 0.0375f;
+  c->mu = 0.95f;
+  c->nesterov = 1;
+  c->ns_steps = 12;
+  c->ns_a = 2.0f;
+  c->ns_b = -1.5f;
+  c->ns_c = 0.5f;
+  c->ns_eps = 1e-7f;
+  c->aurora = 1;
+  c->pp_iterations = 2;
+  c->pp_beta = 0.5f;
+  c->pp_eps = 1e-7f;
+  c->contra = 0.4f;
+  c->power_iters = 5;
+  c->target_uw = 0.35f;
+  c->weight_decay = 0.0f;
+  c->gemm_mode = MUON_GEMM_BF16;
+  c->param_dtype = MUON_BF16;
+  c->grad_dtype = MUON_BF16;
+}
+
+const char* muon_status_string(muon_status s) {
+  switch (s) {
+    case MUON_OK: return "ok";
+    case MUON_ERR_INVALID_ARG: return "invalid argument";
+    case MUON_ERR_UNSUPPORTED: return "unsupported request";
+    case MUON_ERR_WORKSPACE: return "workspace missing or too small";
+    case MUON_ERR_CUDA: return "CUDA error";
+    case MUON_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t muon_workspace_size(const muon_config* cfg, int n, const muon_shape* shapes) {
+  if (!cfg || n <= 0 || !shapes || check_shapes(n, shapes) != MUON_OK) return 0;
+  return make_plan(cfg, n, shapes).total;
+}
+
+muon_status muon_step(const muon_config* cfg, int n, const muon_shape* shapes, void* const* params,
+                      const void* const* grads, float* const* momentum, float* const* update_out,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  muon_status s = check_config(cfg, true, cfg && cfg->aurora, cfg && cfg->contra != 0.f);
+  if (s != MUON_OK) return s;
+  if ((s = check_shapes(n, shapes)) != MUON_OK) return s;
+  if (n == 0) return MUON_OK;
+  if ((s = check_ptrs(n, params, false, false)) != MUON_OK) return s;
+  if ((s = check_ptrs(n, grads, false, false)) != MUON_OK) return s;
+  if ((s = check_ptrs(n, momentum, false, false)) != MUON_OK) return s;
+  if ((s = check_ptrs(n, update_out, true, true)) != MUON_OK) return s;
+  const Plan p = make_plan(cfg, n, shapes);
+  if ((s = check_ws(p, workspace, workspace_bytes)) != MUON_OK) return s;
+
+  Ctx c = make_ctx(cfg, p, workspace, stream);
+  c.W = params;
+  c.G = grads;
+  c.M = momentum;
+  c.V = update_out;
+  const std::vector<int> ids = iota_ids(n);
+  if ((s = stage_prologue(c, ids, 0, cfg->target_uw > 0.f)) != MUON_OK) return s;
+  if (cfg->contra != 0.f && (s = stage_power_iteration(c, ids, cfg->power_iters)) != MUON_OK) return s;
+  if ((s = stage_polar(c, cfg->aurora != 0)) != MUON_OK) return s;
+  if ((s = stage_dots(c, ids)) != MUON_OK) return s;
+  if ((s = set_coeffs(c, ids, 1)) != MUON_OK) return s;
+  return stage_epilogue(c, ids, true, cfg->lr);
+}
+
+static muon_status polar_entry(const muon_config* cfg, int n, const muon_shape* shapes,
+                               const void* const* in, int in_dtype, float* const* out, void* ws,
+                               size_t ws_bytes, void* stream, bool aurora) {
+  muon_status s = check_config(cfg, true, aurora, false);
+  if (s != MUON_OK) return s;
+  if (in_dtype < 0 || in_dtype > 1) return MUON_ERR_INVALID_ARG;
+  if ((s = check_shapes(n, shapes)) != MUON_OK) return s;
+  if (n == 0) return MUON_OK;
+  if ((s = check_ptrs(n, in, false, false)) != MUON_OK) return s;
+  if ((s = check_ptrs(n, out, false, false)) != MUON_OK) return s;
+  const Plan p = make_plan(cfg, n, shapes);
+  if ((s = check_ws(p, ws, ws_bytes)) != MUON_OK) return s;
+  Ctx c = make_ctx(cfg, p, ws, stream);
+  c.V = out;
+  const std::vector<int> ids = iota_ids(n);
+  if ((s = stage_input(c, n, in, in_dtype)) != MUON_OK) return s;
+  if ((s = stage_polar(c, aurora)) != MUON_OK) return s;
+  if ((s = set_coeffs(c, ids, 2)) != MUON_OK) return s;
+  return stage_epilogue(c, ids, false, 0.f);
+}
+
+muon_status ns_polar(const muon_config* cfg, int n, const muon_shape* shapes, const void* const* in,
+                     int in_dtype, float* const* out, void* ws, size_t ws_bytes, void* stream) {
+  return polar_entry(cfg, n, shapes, in, in_dtype, out, ws, ws_bytes, stream, false);
+}
+
+muon_status aurora_polar(const muon_config* cfg, int n, const muon_shape* shapes,
+                         const void* const* in, int in_dtype, float* const* out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  return polar_entry(cfg, n, shapes, in, in_dtype, out, ws, ws_bytes, stream, true);
+}
+
+muon_status opnorm_normalize(const muon_config* cfg, int n, const muon_shape* shapes,
+                             const void* const* in, int in_dtype, float* const* out,
+                             float* sigma_out, void* ws, size_t ws_bytes, void* stream) {
+  muon_status s = check_config(cfg, false, false, true);
+  if (s != MUON_OK) return s;
+  if (in_dtype < 0 || in_dtype > 1) return MUON_ERR_INVALID_ARG;
+  if ((s = check_shapes(n, shapes)) != MUON_OK) return s;
+  if (n == 0) return MUON_OK;
+  if ((s = check_ptrs(n, in, false, false)) != MUON_OK) return s;
+  if ((s = check_ptrs(n, out, true, true)) != MUON_OK) return s;
+  if (sigma_out && !aligned16(sigma_out)) return MUON_ERR_INVALID_ARG;
+  const Plan p = make_plan(cfg, n, shapes);
+  if ((s = check_ws(p, ws, ws_bytes)) != MUON_OK) return s;
+  Ctx c = make_ctx(cfg, p, ws, stream);
+  c.V = out;
+  const std::vector<int> ids = iota_ids(n);
+  if ((s = stage_input(c, n, in, in_dtype)) != MUON_OK) return s;
+  if ((s = stage_power_iteration(c, ids, cfg->power_iters)) != MUON_OK) return s;
+  if (sigma_out) {
+    CK(for_chunks(c, ids, [](const MatDesc&) { return (int64_t)0; }, [&](const MatTable& t, int) {
+      return launch_sigma_out(t, c.scal, sigma_out, c.st);
+    }));
+  }
+  if (out) {
+    if ((s = set_coeffs(c, ids, 3)) != MUON_OK) return s;
+    if ((s = stage_epilogue(c, ids, false, 0.f)) != MUON_OK) return s;
+  }
+  return MUON_OK;
+}
+
+muon_status uw_floor_apply(const muon_config* cfg, int n, const muon_shape* shapes,
+                           const void* const* params, float* const* updates, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (!cfg) return MUON_ERR_INVALID_ARG;
+  if (cfg->param_dtype < 0 || cfg->param_dtype > 1 || !(cfg->target_uw >= 0.f)) return MUON_ERR_INVALID_ARG;
+  muon_status s = check_shapes(n, shapes);
+  if (s != MUON_OK) return s;
+  if (n == 0) return MUON_OK;
+  if ((s = check_ptrs(n, params, false, false)) != MUON_OK) return s;
+  if ((s = check_ptrs(n, updates, false, false)) != MUON_OK) return s;
+  const Plan p = make_plan(cfg, n, shapes);
+  if ((s = check_ws(p, ws, ws_bytes)) != MUON_OK) return s;
+  Ctx c = make_ctx(cfg, p, ws, stream);
+  c.W = const_cast<void* const*>(params);
+  c.V = updates;
+  const std::vector<int> ids = iota_ids(n);
+  auto blocks = [](const MatDesc& d) { return cdiv(d.m * d.n, 4096); };
+  CK(for_chunks(c, ids, blocks, [&](const MatTable& t, int nb) { return launch_sumsq_wv(t, nb, c.partials, c.st); }));
+  CK(for_chunks(c, ids, blocks, [&](const MatTable& t, int) {
+    cudaError_t e = launch_finalize_sums(t, c.partials, 2, S_SUM_U2, S_SUM_W2, c.scal, c.st);
+    if (e != cudaSuccess) return e;
+    return launch_scalars(t, 4, 0, 0.f, 0.f, cfg->target_uw, c.scal, c.st);
+  }));
+  CK(for_chunks(c, ids, blocks, [&](const MatTable& t, int nb) { return launch_scale_v(t, nb, c.scal, c.st); }));
+  return MUON_OK;
+}
+
+void muon_profile_enable(int on) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  if (on) {
+    g_prof.recs.clear();
+    g_prof.used = 0;
+  }
+  g_prof.on = on != 0;
+}
+
+int muon_profile_read(muon_profile_entry* out, int max_entries) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  muon_profile_entry tot[PC_COUNT];
+  std::memset(tot, 0, sizeof(tot));
+  for (int k = 0; k < PC_COUNT; ++k) std::snprintf(tot[k].name, sizeof(tot[k].name), "%s", kProfNames[k]);
+  for (const ProfRecord& r : g_prof.recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return -1;
+    tot[r.cls].launches += 1;
+    tot[r.cls].ms += ms;
+    tot[r.cls].flops += r.flops;
+    tot[r.cls].bytes += r.bytes;
+  }
+  int w = 0;
+  for (int k = 0; k < PC_COUNT && w < max_entries; ++k) out[w++] = tot[k];
+  return w;
+}
+
+muon_status muon_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
+  unsigned int v = 0;
+  if (read_and_clear_device_status(&v) != cudaSuccess) return MUON_ERR_CUDA;
+  return static_cast<muon_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,497 @@
+// Grouped Newton-Schulz GEMMs on the sm_100a tensor cores.
+//
+// Newton-Schulz step ("源码实现", zeropower_via_newtonschulz5 of the Track 3
+// Aurora write-up): A = X X^T, B = b A + c A^2, X' = a X + B X, with bf16
+// operands and fp32 accumulation.
+//
+// Kernel design (persistent, warp-specialised, one CTA per SM):
+//   warp 0      : TMA producer (one lane) -- 128x64 A tile + 256x64 B tile per
+//                 stage, 128-byte swizzle, 4-stage mbarrier ring
+//   warp 1      : TMEM allocator + tcgen05.mma issuer (one lane), M=128 N=256
+//                 K=16 per instruction, fp32 accumulators in TMEM, two
+//                 accumulator buffers (2 x 256 columns) so the epilogue of one
+//                 tile overlaps the main loop of the next
+//   warps 2..5  : epilogue -- tcgen05.ld 32 lanes x 32 columns per warp,
+//                 alpha*acc + beta*E, bf16 stores.  A and A^2 are symmetric:
+//                 only tiles touching the upper triangle run, and each of them
+//                 writes its upper part directly and its strictly-upper part
+//                 mirrored, so every element is written exactly once.
+// Operand majorness: Gram and square read both operands K-major; the update
+// reads X as an MN-major B operand (X is [K][N] with N contiguous).
+// Every mbarrier wait is bounded: on expiry the CTA records MUON_ERR_TIMEOUT,
+// drains its own copies and MMAs (again bounded), frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace am {
+
+// Sticky per-device status word (a muon_status code; the first error wins).
+__device__ unsigned int g_device_status = 0;
+
+namespace {
+
+__device__ __forceinline__ void raise_status(unsigned int code) { atomicCAS(&g_device_status, 0u, code); }
+
+constexpr int TBM = 128, TBN = 256, TBK = 64, STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kABytes = TBM * TBK * 2;           // 16 KiB
+constexpr uint32_t kBBytes = TBN * TBK * 2;           // 32 KiB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * (size_t)kStageBytes + 256;
+constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
+
+struct TcParams {
+  CUtensorMap maps[2 * kMaxGemmGroups];   // per group: operand A, operand B
+  GemmLaunch L;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; returns false (and raises the abort flag) on timeout or when
+// another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(a, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        *abort_flag = 1;
+        raise_status(MUON_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t mbar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and
+// stride byte offsets (all >> 4), version 1, 128-byte swizzle (layout 2).
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, M=128, N=256.
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((uint32_t)(TBN >> 3) << 17) |
+         ((uint32_t)(TBM >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- scheduling
+__device__ __forceinline__ bool symmetric_kind(int kind) { return kind == GK_GRAM || kind == GK_SQR; }
+
+struct TileInfo {
+  int g, b, m0, n0, nkb;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmLaunch& L, int tile) {
+  int g = 0;
+  while (g + 1 < L.num_groups && L.g[g + 1].tile_begin <= tile) ++g;
+  const GemmGroup& G = L.g[g];
+  int t = tile - G.tile_begin;
+  const int b = t / G.tiles_per_mat;
+  t -= b * G.tiles_per_mat;
+  int tm, tn;
+  if (symmetric_kind(G.kind)) {
+    tn = 0;
+    for (;;) {
+      const int cnt = min(2 * tn + 2, G.tiles_m);
+      if (t < cnt) break;
+      t -= cnt;
+      ++tn;
+    }
+    tm = t;
+  } else {
+    tm = t / G.tiles_n;
+    tn = t % G.tiles_n;
+  }
+  TileInfo ti;
+  ti.g = g;
+  ti.b = b;
+  ti.m0 = tm * TBM;
+  ti.n0 = tn * TBN;
+  ti.nkb = (G.K + TBK - 1) / TBK;
+  return ti;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f(uint32_t h) { return __uint_as_float(h << 16); }
+
+// ---------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t sA = base;                         // STAGES x 16 KiB
+  const uint32_t sB = base + STAGES * kABytes;      // STAGES x 32 KiB
+  uint8_t* ctl = smem + STAGES * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);     // full[4], empty[4], tfull[2], tempty[2], drain
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * STAGES;
+  const uint32_t tfull0 = empty0 + 8 * STAGES, tempty0 = tfull0 + 16, drain = tempty0 + 16;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(ctl + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 132);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const GemmLaunch& L = P.L;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < L.num_groups; ++g) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[2 * g])) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[2 * g + 1])) : "memory");
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(const_cast<uint32_t*>(tmem_slot))),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < L.total_tiles && ok; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(L, tile);
+        const GemmGroup& G = L.g[ti.g];
+        const CUtensorMap* mA = &P.maps[2 * ti.g];
+        const CUtensorMap* mB = &P.maps[2 * ti.g + 1];
+        const bool upd = G.kind == GK_UPD;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_expect_tx(fb, kStageBytes);
+          tma_load_3d(sA + stage * kABytes, mA, fb, kb * TBK, ti.m0, ti.b);
+          if (upd) {
+#pragma unroll
+            for (int j = 0; j < TBN / 64; ++j)
+              tma_load_3d(sB + stage * kBBytes + j * (64 * TBK * 2), mB, fb, ti.n0 + 64 * j, kb * TBK, ti.b);
+          } else {
+            tma_load_3d(sB + stage * kBBytes, mB, fb, kb * TBK, ti.n0, ti.b);
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // drain: wait (bounded) for every stage's most recent load to land
+        for (uint32_t k = 0; k < STAGES && k < issued; ++k) {
+          const uint32_t idx = issued - 1 - k;
+          const uint32_t st = idx % STAGES, ph = (idx / STAGES) & 1u;
+          const long long t0 = clock64();
+          while (!mbar_try_wait(full0 + 8 * st, ph) && clock64() - t0 < kWaitLimitCycles) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, any = false;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < L.total_tiles && ok; tile += gridDim.x, ++it) {
+        const TileInfo ti = decode_tile(L, tile);
+        const bool upd = L.g[ti.g].kind == GK_UPD;
+        const uint32_t idesc = make_idesc(upd ? 1u : 0u);
+        const int acc = it & 1;
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TBN);
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = sA + stage * kABytes, b0 = sB + stage * kBBytes;
+#pragma unroll
+          for (int k = 0; k < TBK / 16; ++k) {
+            const uint64_t ad = make_sdesc(a0 + k * 32, 16, 1024);
+            const uint64_t bd = upd ? make_sdesc(b0 + k * 16 * 128, 64 * TBK * 2, 1024)
+                                    : make_sdesc(b0 + k * 32, 16, 1024);
+            tc_mma(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            any = true;
+          }
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        if (acc == 1) acc_phase ^= 1u;
+      }
+      if (!ok && any) {
+        tc_commit(drain);
+        const long long t0 = clock64();
+        while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles) {}
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int r_in_tile = q * 32 + lane;
+    uint32_t acc_phase = 0;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(L, tile);
+      const GemmGroup& G = L.g[ti.g];
+      const int acc = it & 1;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
+      tc_fence_after();
+      float alpha = G.alpha0, beta = G.beta0;
+      if (G.rho) {
+        const float r = G.rho[ti.b];
+        for (int p = 0; p < G.pa; ++p) alpha *= r;
+        for (int p = 0; p < G.pb; ++p) beta *= r;
+      }
+      const int row = ti.m0 + r_in_tile;
+      const bool sym = symmetric_kind(G.kind);
+      __nv_bfloat16* C = reinterpret_cast<__nv_bfloat16*>(G.C) + (int64_t)ti.b * G.sc;
+      const __nv_bfloat16* E =
+          G.E ? reinterpret_cast<const __nv_bfloat16*>(G.E) + (int64_t)ti.b * G.se : nullptr;
+      for (int ch = 0; ch < TBN / 32; ++ch) {
+        const int col0 = ti.n0 + ch * 32;
+        if (col0 >= G.N) break;                                   // warp-uniform
+        if (sym && col0 + 31 < ti.m0) continue;                   // chunk entirely below the diagonal band
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN + ch * 32), r);
+        if (row >= G.M) continue;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
+        const bool full = col0 + 32 <= G.N;
+        if (E) {
+          const __nv_bfloat16* e = E + (int64_t)row * G.lde + col0;
+          if (full) {
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const uint4 w = *reinterpret_cast<const uint4*>(e + 8 * j4);
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                v[8 * j4 + 2 * h] += beta * bf16_bits_to_f(ww[h] & 0xFFFFu);
+                v[8 * j4 + 2 * h + 1] += beta * bf16_bits_to_f(ww[h] >> 16);
+              }
+            }
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < G.N) v[j] += beta * __bfloat162float(e[j]);
+          }
+        }
+        __nv_bfloat16* c = C + (int64_t)row * G.ldc + col0;
+        if (!sym) {
+          if (full) {
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              uint32_t w[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * j4 + 2 * h], v[8 * j4 + 2 * h + 1]);
+                w[h] = *reinterpret_cast<const uint32_t*>(&p);
+              }
+              *reinterpret_cast<uint4*>(c + 8 * j4) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < G.N) c[j] = __float2bfloat16_rn(v[j]);
+          }
+        } else {
+          // direct: col >= row ; mirror: col > row
+#pragma unroll 4
+          for (int j = 0; j < 32; ++j) {
+            const int col = col0 + j;
+            if (col >= G.N) break;
+            if (col >= row) {
+              const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+              c[j] = h;
+              if (col > row) C[(int64_t)col * G.ldc + row] = h;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+      if (acc == 1) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t ld_elems,
+               uint64_t batch_elems, uint32_t box0, uint32_t box1) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {ld_elems * 2, batch_elems * 2};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t read_and_clear_device_status(unsigned int* out) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  *out = v;
+  if (v != 0) e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+  return e;
+}
+
+int tc_tile_count(int kind, int M, int N, int* tiles_m, int* tiles_n) {
+  const int tm = (M + TBM - 1) / TBM, tn = (N + TBN - 1) / TBN;
+  *tiles_m = tm;
+  *tiles_n = tn;
+  if (kind == GK_UPD) return tm * tn;
+  int c = 0;
+  for (int j = 0; j < tn; ++j) c += std::min(2 * j + 2, tm);
+  return c;
+}
+
+bool tc_encode_maps(const GemmLaunch& L, void* maps_out) {
+  CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_out);
+  for (int g = 0; g < L.num_groups; ++g) {
+    const GemmGroup& G = L.g[g];
+    if (!encode_3d(&maps[2 * g], G.A, G.K, G.M, G.count, G.lda, G.sa, TBK, TBM)) return false;
+    bool ok;
+    if (G.kind == GK_UPD)
+      ok = encode_3d(&maps[2 * g + 1], G.B, G.N, G.K, G.count, G.ldb, G.sb, 64, TBK);
+    else
+      ok = encode_3d(&maps[2 * g + 1], G.B, G.K, G.N, G.count, G.ldb, G.sb, TBK, TBN);
+    if (!ok) return false;
+  }
+  return true;
+}
+
+cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, cudaStream_t st) {
+  if (L.total_tiles == 0) return cudaSuccess;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  TcParams* P = new TcParams;
+  std::memcpy(P->maps, maps, sizeof(CUtensorMap) * 2 * L.num_groups);
+  P->L = L;
+  const int grid = std::min(num_sms, L.total_tiles);
+  k_gemm_tc<<<grid, kThreads, kSmemBytes, st>>>(*P);
+  delete P;
+  return cudaGetLastError();
+}
+
+}  // namespace am

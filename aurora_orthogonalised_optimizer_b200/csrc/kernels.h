@@ -1,0 +1,77 @@
+// Internal launch interface between the host engine and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace am {
+
+// ---------------------------------------------------------------- GEMM groups
+// One group = one shape bucket of `count` same-shape matrices stored as a
+// batched tensor [count][rows][ld].  All operands use the Newton-Schulz dtype.
+enum GemmKind {
+  GK_GRAM = 0,   // C[s x s] = alpha * X X^T          (A = X, B = X, K = l)
+  GK_SQR = 1,    // C[s x s] = alpha * A A + beta * E (E = A), symmetric A
+  GK_UPD = 2     // C[s x l] = alpha * B X + beta * E (E = X), K = s
+};
+
+struct GemmGroup {
+  int kind;
+  int count;
+  int M, N, K;
+  int tiles_m, tiles_n, tiles_per_mat;
+  int tile_begin;                 // first tile of this group in the launch
+  const void* A; int64_t lda, sa; // operand A: [count][M][lda], K contiguous
+  const void* B; int64_t ldb, sb; // operand B: GRAM/SQR: [count][N][ldb] (K contiguous);
+                                  //            UPD: [count][K][ldb] (N contiguous)
+  void* C; int64_t ldc, sc;
+  const void* E; int64_t lde, se; // epilogue addend (may be null)
+  const float* rho;               // per-batch normalisation scale (may be null)
+  float alpha0, beta0;            // alpha = alpha0 * rho^pa, beta = beta0 * rho^pb
+  int pa, pb;
+};
+
+constexpr int kMaxGemmGroups = 16;
+
+struct GemmLaunch {
+  int num_groups;
+  int total_tiles;
+  int dtype;                      // kF32 or kBF16
+  GemmGroup g[kMaxGemmGroups];
+};
+
+// SIMT grouped GEMM (fp32 FMA accumulation; bf16 or fp32 storage).
+cudaError_t launch_gemm_simt(const GemmLaunch& L, cudaStream_t st);
+
+// tcgen05 grouped GEMM (bf16 operands, fp32 accumulation in TMEM, TMA loads).
+// `maps` holds two CUtensorMap (128 B each) per group: operand A, operand B.
+struct TcLaunch;
+cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, cudaStream_t st);
+bool tc_encode_maps(const GemmLaunch& L, void* maps_out);  // host: builds the tensor maps
+int tc_tile_count(int kind, int M, int N, int* tiles_m, int* tiles_n);
+cudaError_t read_and_clear_device_status(unsigned int* out);  // current device
+
+// ---------------------------------------------------------------- element-wise
+cudaError_t launch_prologue(const MatTable& t, int nblk, int mode, float mu, int nesterov,
+                            int want_w2, double* partials, cudaStream_t st);
+cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int nq, int slot0,
+                                 int slot1, double* scal, cudaStream_t st);
+cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, float beta,
+                           cudaStream_t st);
+cudaError_t launch_scale_cols(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+cudaError_t launch_scalars(const MatTable& t, int op, int src_slot, float ns_eps, float contra,
+                           float target_uw, double* scal, cudaStream_t st);
+cudaError_t launch_matvec(const MatTable& t, int nblk, int dir, cudaStream_t st);
+cudaError_t launch_vecop(const MatTable& t, int which, int mode, int len_is_s_when_flag0,
+                         double* scal, cudaStream_t st);
+cudaError_t launch_dots(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
+                            cudaStream_t st);
+cudaError_t launch_sumsq_wv(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+cudaError_t launch_scale_v(const MatTable& t, int nblk, const double* scal, cudaStream_t st);
+cudaError_t launch_copy_rho(const MatTable& t, const double* scal, cudaStream_t st);
+cudaError_t launch_sigma_out(const MatTable& t, const double* scal, float* sigma_out, cudaStream_t st);
+
+}  // namespace am

@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon / Aurora optimizer step on B200.
+
+One step = one full optimizer step (momentum + Nesterov, power iteration,
+Aurora-equilibrated Newton-Schulz polar, contra subtraction and Frobenius
+restore, aspect scale, u/w floor, parameter add) over every 2-D matrix of the
+workload, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   (the float64 CPU oracle, same metric)
+
+Default workload: the 3.8B Llama-style matrix set (28 layers, 168 matrices,
+2.82 G parameters) with the full Aurora + Contra-Muon + u/w-floor stack,
+bf16 params/grads, fp32 momentum.  Inputs are synthetic (seeded) and larger
+than L2, so no flush is needed between steps.  For N > 1 (torchrun) the
+matrices are sharded by LPT over ranks and one NCCL all-gather of the
+updated parameters closes each step (strong scaling).  Rank 0 prints one
+JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = "Muon/Aurora steps/s & NS TFLOP/s (% bf16 peak) on 3.8B matrix shapes"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama_aurora", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=28, help="layers of the 3.8B set (28 = full)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm", default="bf16", choices=["bf16", "fp32", "bf16simt"])
+    return ap.parse_args()
+
+
+def make_workload(args):
+    if args.workload in ("llama_plain", "llama_aurora"):
+        return WL.WORKLOADS[args.workload](layers=args.layers)
+    return WL.WORKLOADS[args.workload]()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def nominal_ns_flops(wl) -> float:
+    c = wl.cfg
+    tot = 0.0
+    for m, n in wl.shapes:
+        s, l = min(m, n), max(m, n)
+        polars = c.pp_iterations if (c.aurora and m != n) else 1
+        tot += polars * c.ns_steps * (4.0 * s * s * l + 2.0 * s ** 3)
+    return tot
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample_time(wl, indices):
+    """Wall time of the float64 oracle stepping `indices` of the workload once."""
+    import oracle.muon_oracle as O
+    Ws, Gs, Ms = WL.generate(wl, indices)
+    t0 = time.perf_counter()
+    for k, i in enumerate(indices):
+        O.step(WL.to_f64(Ws[k], wl.param_dtype), WL.to_f64(Gs[k], wl.grad_dtype), Ms[k].astype(np.float64),
+               wl.cfg, wl.param_dtype)
+    return time.perf_counter() - t0
+
+
+def sample_indices(wl):
+    if wl.name.startswith("llama"):
+        return [0, 1, 2]                       # layer 0: q (3072^2), k, v (1024 x 3072)
+    if wl.n <= 8:
+        return list(range(wl.n))
+    return [0, 1]
+
+
+def sample_flops(wl, idx):
+    sub = WL.Workload(wl.name, wl.seed, [wl.shapes[i] for i in idx], wl.param_dtype, wl.grad_dtype,
+                      [wl.w_std[i] for i in idx], wl.grad_kind, wl.grad_base, wl.grad_sigma, wl.cfg, 1)
+    return nominal_ns_flops(sub)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([d.get("num_threads", 1) for d in info] or [os.cpu_count() or 1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, reps=1):
+    idx = sample_indices(wl)
+    t = min(oracle_sample_time(wl, idx) for _ in range(reps))
+    scale = nominal_ns_flops(wl) / max(sample_flops(wl, idx), 1.0)
+    step_s = t * scale
+    names = ",".join(f"{wl.shapes[i][0]}x{wl.shapes[i][1]}" for i in idx)
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(idx)} of {wl.n} matrices ({names}) stepped by the float64 NumPy oracle in "
+                      f"{t:.2f} s, scaled to the whole step by nominal Newton-Schulz FLOPs (x{scale:.1f})"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = make_workload(args)
+    idx = sample_indices(wl)
+    scale = nominal_ns_flops(wl) / max(sample_flops(wl, idx), 1.0)
+    for _ in range(args.warmup):
+        oracle_sample_time(wl, idx)
+    ts = [oracle_sample_time(wl, idx) for _ in range(args.steps)]
+    step_s = sum(ts) / len(ts) * scale
+    v = 1.0 / step_s
+    names = ",".join(f"{wl.shapes[i][0]}x{wl.shapes[i][1]}" for i in idx)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "matrices": wl.n, "elements": wl.elements()},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: {len(idx)} of {wl.n} matrices ({names}), scaled by nominal "
+                                   f"Newton-Schulz FLOPs (x{scale:.1f})"},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU leg
+def traffic_record(kernel_src):
+    """Per-launch DRAM traffic from the committed ncu summary, if taken on this exact kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+        if d.get("source_sha256_16") != h:
+            return None
+        return d
+    except Exception:
+        return None
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from aurora_orthogonalised_optimizer_b200 import _abi as A
+    from aurora_orthogonalised_optimizer_b200 import sharding as SH
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    wl = make_workload(args)
+    gemm = {"bf16": A.MUON_GEMM_BF16, "fp32": A.MUON_GEMM_FP32, "bf16simt": A.MUON_GEMM_BF16_SIMT}[args.gemm]
+    cfg = A.Config.from_step_config(wl.cfg, gemm_mode=gemm,
+                                    param_dtype=1 if wl.param_dtype == WL.BF16 else 0,
+                                    grad_dtype=1 if wl.grad_dtype == WL.BF16 else 0)
+    shapes = wl.shapes
+    costs = SH.step_costs(shapes, wl.cfg.ns_steps, wl.cfg.aurora, wl.cfg.pp_iterations)
+    owned_all = SH.lpt_partition(costs, world)
+    owned = owned_all[rank]
+    layout = SH.flat_layout(shapes, owned_all)
+    pdt = torch.bfloat16 if wl.param_dtype == WL.BF16 else torch.float32
+    gdt = torch.bfloat16 if wl.grad_dtype == WL.BF16 else torch.float32
+
+    # ---- inputs: every rank holds all params (flat, sharded layout); grads and momentum of its own matrices
+    threads = min(32, os.cpu_count() or 8)
+    flat = torch.empty(layout.total_elems, dtype=pdt, device=dev)
+    pviews = SH.views(flat, layout, shapes)
+    W_host, G_host = WL.generate_torch(wl, owned, 0, threads)
+    for k, i in enumerate(owned):
+        pviews[i].copy_(W_host[k])
+    if world > 1:
+        SH.exchange(flat, layout, rank)
+    params = [pviews[i] for i in owned]
+    grads = [G_host[k].to(dev) for k in range(len(owned))]
+    mom = [torch.zeros(shapes[i], dtype=torch.float32, device=dev) for i in owned]
+    my_shapes = [shapes[i] for i in owned]
+    ws = A.make_workspace(cfg, my_shapes, dev)
+    del W_host
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        A.muon_step(cfg, params, grads, mom, None, ws, stream)
+        if world > 1:
+            SH.exchange(flat, layout, rank)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if A.last_device_status(stream) != A.MUON_OK:
+        raise SystemExit("device status error during warm-up")
+
+    # ---- timed region (device time, CUDA events on the launch stream)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
+    A.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    A.profile_enable(False)
+    prof = A.profile_read()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    steps_per_s = 1e3 / ms_per_step
+
+    # ---- end to end: grads host->device from pinned memory, step, params device->host
+    e2e = None
+    if not args.no_e2e:
+        g_pin = [G_host[k].pin_memory() for k in range(len(owned))]
+        p_pin = [torch.empty(shapes[i], dtype=pdt).pin_memory() for i in owned]
+        h2d = sum(t.numel() * t.element_size() for t in g_pin)
+        d2h = sum(t.numel() * t.element_size() for t in p_pin)
+        barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            for k in range(len(owned)):
+                grads[k].copy_(g_pin[k], non_blocking=True)
+            step()
+            for k in range(len(owned)):
+                p_pin[k].copy_(params[k], non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": 1e3 * args.steps / ems, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+        if world > 1:
+            tot = torch.tensor([h2d, d2h], dtype=torch.float64, device=dev)
+            dist.all_reduce(tot)
+            e2e["h2d_bytes_per_step"], e2e["d2h_bytes_per_step"] = int(tot[0].item()), int(tot[1].item())
+
+    if A.last_device_status(stream) != A.MUON_OK:
+        raise SystemExit("device status error in the timed region")
+
+    # ---- roofline of the dominant kernel + per-stage figures
+    peaks, peak_kind = load_peaks()
+    gk = "ns_gemm_tc" if gemm == A.MUON_GEMM_BF16 else "ns_gemm_simt"
+    g = prof.get(gk, {"launches": 0, "ms": 0.0, "flops": 0.0})
+    launches = sum(v["launches"] for v in prof.values())
+    achieved_tf = g["flops"] / max(g["ms"], 1e-9) / 1e9  # flops / ms -> TFLOP/s
+    peak_tf = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    tr = traffic_record(os.path.join(ROOT, "aurora_orthogonalised_optimizer_b200", "csrc", "gemm_tc.cu"))
+    traffic = None
+    if tr is not None and g["launches"]:
+        traffic = tr.get("bytes_per_flop", 0.0) * g["flops"] / g["launches"]
+    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved_tf / peak_tf, "traffic": traffic,
+                "kernel": "k_gemm_tc" if gk == "ns_gemm_tc" else "k_gemm_simt",
+                "peak_kind": f"bf16_tflops_sustained ({peak_kind})",
+                "flops_per_launch": g["flops"] / max(1, g["launches"]),
+                "ms_per_launch": g["ms"] / max(1, g["launches"])}
+    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    stages = {}
+    for k, v in prof.items():
+        if v["launches"] == 0:
+            continue
+        st = {"launches": v["launches"] // args.steps, "ms_per_step": v["ms"] / args.steps,
+              "share": v["ms"] / max(sum(x["ms"] for x in prof.values()), 1e-9)}
+        if v["bytes"] > 0:
+            st["GB/s"] = v["bytes"] / v["ms"] / 1e6
+            st["frac_hbm"] = st["GB/s"] / hbm
+        if v["flops"] > 0:
+            st["TFLOP/s"] = v["flops"] / v["ms"] / 1e9
+        stages[k] = st
+    ns_nominal = nominal_ns_flops(wl)
+    ns_tf_nominal = ns_nominal * steps_per_s / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16" if gemm != A.MUON_GEMM_FP32 else "f32",
+            "data": "synthetic (seeded N(0,1) grads x 1e-3 with log-normal(0,0.5) row scales, N(0,1/fan_in) "
+                    "weights)" if wl.name.startswith("llama") else "synthetic (seeded)",
+            "config": {"workload": wl.name, "matrices": wl.n, "elements": wl.elements(),
+                       "parallelism": f"matrix-sharded x{world} (LPT) + all-gather" if world > 1 else "single GPU",
+                       "gemm": args.gemm, "l2": "inputs (>20 GB) larger than the 126 MB L2; no flush"},
+            "matrices_per_s": wl.n * steps_per_s,
+            "ns_tflops_nominal": ns_tf_nominal,
+            "ns_frac_of_peak_nominal": ns_tf_nominal / peak_tf,
+            "roofline": roofline,
+            "stages": stages,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -241,3 +241,50 @@ def grads(wl: Workload, step: int, indices: Optional[Sequence[int]] = None, thre
         with ThreadPoolExecutor(threads) as ex:
             return list(ex.map(lambda i: grad(wl, i, step), idx))
     return [grad(wl, i, step) for i in idx]
+
+
+# --------------------------------------------------------------------------
+# fast path for large workloads: the same float32 draws, cast to the storage
+# dtype by torch on the CPU (round-to-nearest-even, identical values to
+# f32_to_bf16_bits), returned as torch CPU tensors.
+# --------------------------------------------------------------------------
+def _draw_w32(wl: Workload, idx: int) -> np.ndarray:
+    m, n = wl.shapes[idx]
+    x = _rng(wl.seed, idx, 0, STREAM_W).standard_normal((m, n), dtype=np.float32)
+    x *= np.float32(wl.w_std[idx])
+    return x
+
+
+def _draw_g32(wl: Workload, idx: int, step: int) -> np.ndarray:
+    m, n = wl.shapes[idx]
+    x = _rng(wl.seed, idx, step, STREAM_G).standard_normal((m, n), dtype=np.float32)
+    srng = _rng(wl.seed, idx, 0, STREAM_SCALE)
+    if wl.grad_kind == "matrix_scale":
+        x *= np.float32(10.0 ** srng.uniform(-4.0, -1.0))
+    elif wl.grad_kind == "row_lognormal":
+        r = np.exp(wl.grad_sigma * srng.standard_normal(m)).astype(np.float32)
+        x *= r[:, None]
+    if wl.grad_base != 1.0:
+        x *= np.float32(wl.grad_base)
+    return x
+
+
+def _to_torch(x32: np.ndarray, dtype: str):
+    import torch
+    t = torch.from_numpy(x32)
+    return t.to(torch.bfloat16) if dtype == BF16 else t
+
+
+def generate_torch(wl: Workload, indices: Optional[Sequence[int]] = None, step: int = 0, threads: int = 8,
+                   want_w: bool = True, want_g: bool = True):
+    """(W list, G list) as torch CPU tensors in their storage dtypes."""
+    idx = list(range(wl.n)) if indices is None else list(indices)
+
+    def one(i):
+        w = _to_torch(_draw_w32(wl, i), wl.param_dtype) if want_w else None
+        g = _to_torch(_draw_g32(wl, i, step), wl.grad_dtype) if want_g else None
+        return w, g
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        res = list(ex.map(one, idx))
+    return [r[0] for r in res], [r[1] for r in res]
