@@ -23,7 +23,7 @@ MUON_GEMM_BF16, MUON_GEMM_FP32, MUON_GEMM_BF16_SIMT = 0, 1, 2
 
 EXPORTS = ["muon_config_default", "muon_workspace_size", "muon_step", "ns_polar", "aurora_polar",
            "opnorm_normalize", "uw_floor_apply", "muon_last_device_status", "muon_status_string",
-           "muon_profile_enable", "muon_profile_read"]
+           "muon_profile_enable", "muon_profile_read", "opnorm_normalize_noalloc"]
 
 
 class MuonShape(C.Structure):
@@ -81,6 +81,9 @@ def load():
     lib.opnorm_normalize.argtypes = [C.POINTER(MuonConfig), C.c_int, C.POINTER(MuonShape), PP, C.c_int, PP,
                                      P, P, C.c_size_t, P]
     lib.opnorm_normalize.restype = C.c_int
+    lib.opnorm_normalize_noalloc.argtypes = [C.POINTER(MuonConfig), C.c_int, C.POINTER(MuonShape), PP, C.c_int,
+                                             PP, P, P]
+    lib.opnorm_normalize_noalloc.restype = C.c_int
     lib.uw_floor_apply.argtypes = [C.POINTER(MuonConfig), C.c_int, C.POINTER(MuonShape), PP, PP, P,
                                    C.c_size_t, P]
     lib.uw_floor_apply.restype = C.c_int
@@ -245,6 +248,22 @@ def opnorm_normalize(cfg: Config, inputs: List, outputs: Optional[List], sigma_o
                                    wp, wb, _stream(stream))
     if check:
         _raise(code, "opnorm_normalize")
+    return code
+
+
+def opnorm_normalize_noalloc(cfg: Config, inputs: List, outputs: Optional[List], sigma_out=None, stream=None,
+                             check: bool = True) -> int:
+    """opnorm_normalize without a workspace, for callers that cannot allocate
+    device memory at this point; scratch is the library's static 1 MiB array."""
+    n = len(inputs)
+    shapes = [tuple(t.shape) for t in inputs]
+    dt = dtype_code(inputs[0]) if n else MUON_F32
+    code = load().opnorm_normalize_noalloc(C.byref(cfg.to_c()), n, _shapes(shapes), _ptrs(inputs, n), dt,
+                                           _ptrs(outputs, n),
+                                           None if sigma_out is None else int(sigma_out.data_ptr()),
+                                           _stream(stream))
+    if check:
+        _raise(code, "opnorm_normalize_noalloc")
     return code
 
 

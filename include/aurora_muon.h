@@ -137,6 +137,30 @@ muon_status opnorm_normalize(const muon_config* cfg, int n, const muon_shape* sh
                              float* sigma_out, void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* Workspace-free variant of opnorm_normalize (the pages have no counterpart;
+ * it exists for callers that cannot allocate device memory where they need
+ * this step: code under a framework whose memory manager owns the whole
+ * device, or loops that must not enter the allocator after start-up).
+ * Same results as opnorm_normalize within rounding: sigma = |A v| after
+ * cfg->power_iters steps of v <- A^T A v / |A^T A v| from ones(n)/sqrt(n),
+ * out = A / max(sigma, 1e-10), computed directly on the input in its own
+ * dtype (in_dtype) and orientation.  Uses cfg->power_iters only.
+ *  - Scratch: a 1 MiB file-scope device array inside the library (held by
+ *    every GPU that loads the library until exit).  A call needs
+ *    n * 128 bytes plus 4 * (round_up(rows, 64) + round_up(cols, 64)) bytes
+ *    per matrix; larger requests return MUON_ERR_UNSUPPORTED before
+ *    anything is launched.
+ *  - Calls no cudaMalloc / cudaFree.  The first call on a device looks up
+ *    the array's device address (cudaGetSymbolAddress, with that device
+ *    current); make that first call before any stream capture.
+ *  - Every call shares the one array and it keeps the last call's contents;
+ *    each call clears its scalar block first.  Calls that overlap on the
+ *    GPU (different streams, or different host threads on one device) race
+ *    on the array: serialise them. */
+muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, const muon_shape* shapes,
+                                     const void* const* in, int in_dtype, float* const* out,
+                                     float* sigma_out, void* stream);
+
 /* u/w floor ("u/w-floor"): for each matrix, with p = max(|W|_F, 1e-8) and
  * q = max(|U|_F, 1e-8), if q / p < cfg->target_uw the fp32 update U is
  * scaled in place by target_uw * p / q.  params are read only (param_dtype
