@@ -359,7 +359,7 @@ double gemm_flops(const GemmLaunch& L) {
 muon_status gemm_launch(const Ctx& c, GemmLaunch& L) {
   if (L.num_groups == 0) return MUON_OK;
   if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
-    alignas(64) unsigned char maps[kMaxGemmGroups * 2 * 128];
+    alignas(64) unsigned char maps[kMaxGemmGroups * 3 * 128];
     if (!tc_encode_maps(L, maps)) return MUON_ERR_CUDA;
     ProfScope ps(PC_GEMM_TC, gemm_flops(L), 0.0, c.st);
     CK(launch_gemm_tc(L, maps, num_sms_current(), c.st));
@@ -386,19 +386,36 @@ void add_group(const Ctx& c, GemmLaunch& L, GemmGroup g) {
 }
 
 // ns_steps Newton-Schulz iterations on every matrix of the given buckets.
-// it = 0 reads X0 (uX, or Q when x0_in_Q) scaled by rho; output ping-pongs
-// P (even it), Q (odd it).
-muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids, bool x0_in_Q) {
+// it = 0 reads X0 scaled by rho: uX, or Q for the buckets flagged in
+// x0_in_Q (Aurora's D-scaled input); the iterates ping-pong P (even it),
+// Q (odd it).
+muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids_in,
+                                const std::vector<bool>& x0_in_Q_in) {
   const Plan& p = *c.plan;
   const float a = c.cfg->ns_a, bc = c.cfg->ns_b, cc = c.cfg->ns_c;
+  // Longest tiles first: the persistent kernel deals tiles round-robin in
+  // group order, so big-K groups up front shorten the launch's tail.
+  std::vector<size_t> order(bucket_ids_in.size());
+  for (size_t k = 0; k < order.size(); ++k) order[k] = k;
+  std::stable_sort(order.begin(), order.end(), [&](size_t x, size_t y) {
+    const BucketPlan& bx = p.buckets[bucket_ids_in[x]];
+    const BucketPlan& by = p.buckets[bucket_ids_in[y]];
+    return bx.s != by.s ? bx.s > by.s : bx.l > by.l;
+  });
+  std::vector<int> bucket_ids;
+  std::vector<bool> x0_in_Q;
+  for (size_t k : order) {
+    bucket_ids.push_back(bucket_ids_in[k]);
+    x0_in_Q.push_back(x0_in_Q_in[k]);
+  }
   for (int it = 0; it < c.cfg->ns_steps; ++it) {
     for (int kind = 0; kind < 3; ++kind) {
       GemmLaunch L;
       std::memset(&L, 0, sizeof(L));
       L.dtype = p.ns_dtype;
-      for (int bi : bucket_ids) {
-        const BucketPlan& b = p.buckets[bi];
-        char* X_in = c.ws + (it == 0 ? (x0_in_Q ? b.off_Q : b.off_uX) : ((it & 1) ? b.off_P : b.off_Q));
+      for (size_t k = 0; k < bucket_ids.size(); ++k) {
+        const BucketPlan& b = p.buckets[bucket_ids[k]];
+        char* X_in = c.ws + (it == 0 ? (x0_in_Q[k] ? b.off_Q : b.off_uX) : ((it & 1) ? b.off_P : b.off_Q));
         char* X_out = c.ws + ((it & 1) ? b.off_Q : b.off_P);
         char* Ab = c.ws + b.off_A;
         char* Bb = c.ws + b.off_B;
@@ -450,39 +467,37 @@ std::vector<int> ids_of_buckets(const Plan& p, const std::vector<int>& bids) {
 }
 
 // Polar factor of u (in X orientation) for every matrix; result in UX.
+// Square matrices (and every matrix without Aurora) take one plain polar of
+// u; with Aurora the non-square ones take pp_iterations polars of D-scaled u.
+// The first polar of both kinds runs in the same grouped launches.
 muon_status stage_polar(const Ctx& c, bool aurora) {
   const Plan& p = *c.plan;
-  std::vector<int> all_b, sq_b, ns_b;
-  for (int b = 0; b < (int)p.buckets.size(); ++b) {
-    all_b.push_back(b);
-    (p.buckets[b].s == p.buckets[b].l ? sq_b : ns_b).push_back(b);
-  }
-  const std::vector<int> plain_b = aurora ? sq_b : all_b;
+  std::vector<int> plain_b, eq_b;
+  for (int b = 0; b < (int)p.buckets.size(); ++b)
+    ((aurora && p.buckets[b].s != p.buckets[b].l) ? eq_b : plain_b).push_back(b);
   const float eps = c.cfg->ns_eps;
-  if (!plain_b.empty()) {
-    std::vector<int> ids = ids_of_buckets(p, plain_b);
-    CK(for_chunks(c, ids, [](const MatDesc&) { return (int64_t)0; }, [&](const MatTable& t, int) {
+  const float pe = c.cfg->pp_eps, beta = c.cfg->pp_beta;
+  const std::vector<int> plain_ids = ids_of_buckets(p, plain_b), eq_ids = ids_of_buckets(p, eq_b);
+  if (!plain_ids.empty())
+    CK(for_chunks(c, plain_ids, [](const MatDesc&) { return (int64_t)0; }, [&](const MatTable& t, int) {
       ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
       cudaError_t e = launch_scalars(t, 0, S_SUM_U2, eps, 0.f, 0.f, c.scal, c.st);
       if (e != cudaSuccess) return e;
       return launch_copy_rho(t, c.scal, c.st);
     }));
-    muon_status s = stage_newton_schulz(c, plain_b, false);
-    if (s != MUON_OK) return s;
-  }
-  if (aurora && !ns_b.empty()) {
-    std::vector<int> ids = ids_of_buckets(p, ns_b);
-    const float pe = c.cfg->pp_eps, beta = c.cfg->pp_beta;
-    CK(for_chunks(c, ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
+  if (!eq_ids.empty())
+    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
       ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
       return launch_colnorm(t, nb, 0, pe, beta, c.st);
     }));
-    for (int k = 0; k < c.cfg->pp_iterations; ++k) {
-      CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int nb) {
+  const int rounds = eq_b.empty() ? 1 : c.cfg->pp_iterations;
+  for (int k = 0; k < rounds; ++k) {
+    if (!eq_ids.empty()) {
+      CK(for_chunks(c, eq_ids, tiles_x, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
         return launch_scale_cols(t, nb, c.partials, c.st);
       }));
-      CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int) {
+      CK(for_chunks(c, eq_ids, tiles_x, [&](const MatTable& t, int) {
         ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
         cudaError_t e = launch_finalize_sums(t, c.partials, 1, S_SUM_X02, -1, c.scal, c.st);
         if (e != cudaSuccess) return e;
@@ -490,14 +505,18 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
         if (e != cudaSuccess) return e;
         return launch_copy_rho(t, c.scal, c.st);
       }));
-      muon_status s = stage_newton_schulz(c, ns_b, true);
-      if (s != MUON_OK) return s;
-      if (k < c.cfg->pp_iterations - 1)
-        CK(for_chunks(c, ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
-          ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
-          return launch_colnorm(t, nb, 1, pe, beta, c.st);
-        }));
     }
+    std::vector<int> bids = eq_b;
+    std::vector<bool> in_q(eq_b.size(), true);
+    if (k == 0)
+      for (int b : plain_b) { bids.push_back(b); in_q.push_back(false); }
+    muon_status s = stage_newton_schulz(c, bids, in_q);
+    if (s != MUON_OK) return s;
+    if (k < rounds - 1)
+      CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
+        ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
+        return launch_colnorm(t, nb, 1, pe, beta, c.st);
+      }));
   }
   return MUON_OK;
 }

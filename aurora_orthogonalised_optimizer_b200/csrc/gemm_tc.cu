@@ -44,11 +44,13 @@ constexpr uint32_t kABytes = TBM * TBK * 2;           // 16 KiB
 constexpr uint32_t kBBytes = TBN * TBK * 2;           // 32 KiB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * (size_t)kStageBytes + 256;
+constexpr uint32_t kOutTileBytes = 32 * 32 * 2;        // one staged 32x32 bf16 output block
+constexpr uint32_t kOutBytes = 4 /*warps*/ * 4 /*2 parities x {direct, mirror}*/ * kOutTileBytes;
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * (size_t)kStageBytes + kOutBytes + 256;
 constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 
 struct TcParams {
-  CUtensorMap maps[2 * kMaxGemmGroups];   // per group: operand A, operand B
+  CUtensorMap maps[3 * kMaxGemmGroups];   // per group: operand A, operand B, output C
   GemmLaunch L;
 };
 
@@ -130,6 +132,48 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t a, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
+}
+__device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
+  return v;
+}
+// Byte offset of (row r, byte b) inside a 32 x 64-byte block stored with the
+// TMA 64-byte swizzle: 16-byte chunk index XOR ((r >> 1) & 3).
+__device__ __forceinline__ uint32_t swz64(int r, int b) {
+  return (uint32_t)(r * 64 + ((((b >> 4) ^ (r >> 1)) & 3) << 4) + (b & 15));
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 32 consecutive bf16 of one row of E (cols col0.., masked to < N) -> 4 x uint4.
+__device__ __forceinline__ void load_e_chunk(const __nv_bfloat16* erow, int col0, int N, uint4 (&out)[4]) {
+  const __nv_bfloat16* e = erow + col0;
+  if (col0 + 32 <= N) {
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) out[j4] = __ldg(reinterpret_cast<const uint4*>(e) + j4);
+  } else {
+    uint32_t w[16] = {};
+    for (int j = 0; j < 32 && col0 + j < N; ++j) {
+      const uint32_t h = __bfloat16_as_ushort(e[j]);
+      w[j >> 1] |= h << (16 * (j & 1));
+    }
+    for (int j4 = 0; j4 < 4; ++j4) out[j4] = make_uint4(w[4 * j4], w[4 * j4 + 1], w[4 * j4 + 2], w[4 * j4 + 3]);
+  }
+}
+
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
 // stride byte offsets (all >> 4), version 1, 128-byte swizzle (layout 2).
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -194,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sA = base;                         // STAGES x 16 KiB
   const uint32_t sB = base + STAGES * kABytes;      // STAGES x 32 KiB
-  uint8_t* ctl = smem + STAGES * kStageBytes;
+  const uint32_t sOut = sB + STAGES * kBBytes;       // 32 KiB of output staging
+  uint8_t* ctl = smem + STAGES * kStageBytes + kOutBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);     // full[4], empty[4], tfull[2], tempty[2], drain
   const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * STAGES;
   const uint32_t tfull0 = empty0 + 8 * STAGES, tempty0 = tfull0 + 16, drain = tempty0 + 16;
@@ -220,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   }
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < L.num_groups; ++g) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[2 * g])) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[2 * g + 1])) : "memory");
+      for (int k = 0; k < 3; ++k)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[3 * g + k])) : "memory");
     }
   }
   if (warp == 1) {
@@ -246,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       for (int tile = blockIdx.x; tile < L.total_tiles && ok; tile += gridDim.x) {
         const TileInfo ti = decode_tile(L, tile);
         const GemmGroup& G = L.g[ti.g];
-        const CUtensorMap* mA = &P.maps[2 * ti.g];
-        const CUtensorMap* mB = &P.maps[2 * ti.g + 1];
+        const CUtensorMap* mA = &P.maps[3 * ti.g];
+        const CUtensorMap* mB = &P.maps[3 * ti.g + 1];
         const bool upd = G.kind == GK_UPD;
         for (int kb = 0; kb < ti.nkb; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -317,9 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                  // TMEM lane quadrant of this warp
-    const int r_in_tile = q * 32 + lane;
-    uint32_t acc_phase = 0;
+    // Each warp owns 32 rows (its TMEM lane quadrant) and walks the tile in
+    // 32-column chunks: TMEM -> registers -> alpha*acc + beta*E -> bf16 ->
+    // a 32x32 block staged in shared memory (64-byte swizzle) -> TMA store.
+    // Symmetric kinds also store the transposed block (mirror); the block on
+    // the diagonal is completed from its own upper triangle in shared memory.
+    const int q = warp & 3;                          // TMEM lane quadrant of this warp
+    const uint32_t wbuf = sOut + (uint32_t)(warp - 2) * 4u * kOutTileBytes;
+    uint32_t acc_phase = 0, par = 0;
     int it = 0;
     for (int tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x, ++it) {
       const TileInfo ti = decode_tile(L, tile);
@@ -333,75 +383,85 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         for (int p = 0; p < G.pa; ++p) alpha *= r;
         for (int p = 0; p < G.pb; ++p) beta *= r;
       }
-      const int row = ti.m0 + r_in_tile;
+      const int r0 = ti.m0 + q * 32;                 // first row of this warp's strip
+      const int row = r0 + lane;
       const bool sym = symmetric_kind(G.kind);
-      __nv_bfloat16* C = reinterpret_cast<__nv_bfloat16*>(G.C) + (int64_t)ti.b * G.sc;
-      const __nv_bfloat16* E =
-          G.E ? reinterpret_cast<const __nv_bfloat16*>(G.E) + (int64_t)ti.b * G.se : nullptr;
-      for (int ch = 0; ch < TBN / 32; ++ch) {
+      const CUtensorMap* mC = &P.maps[3 * ti.g + 2];
+      const __nv_bfloat16* Erow =
+          (G.E && row < G.M) ? reinterpret_cast<const __nv_bfloat16*>(G.E) + (int64_t)ti.b * G.se +
+                                   (int64_t)row * G.lde
+                             : nullptr;
+      // chunk ch is needed when it is inside N and (symmetric) not below the diagonal
+      auto wanted = [&](int ch) {
+        const int c0 = ti.n0 + ch * 32;
+        return r0 < G.M && c0 < G.N && !(sym && c0 < r0);
+      };
+      uint4 en[4] = {};
+      int next = 0;
+      while (next < TBN / 32 && !wanted(next)) ++next;
+      if (next < TBN / 32 && Erow) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
+      while (next < TBN / 32) {
+        const int ch = next;
         const int col0 = ti.n0 + ch * 32;
-        if (col0 >= G.N) break;                                   // warp-uniform
-        if (sym && col0 + 31 < ti.m0) continue;                   // chunk entirely below the diagonal band
+        const uint4 ec[4] = {en[0], en[1], en[2], en[3]};
+        ++next;
+        while (next < TBN / 32 && !wanted(next)) ++next;
+        if (next < TBN / 32 && Erow) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN + ch * 32), r);
-        if (row >= G.M) continue;
-        float v[32];
+        uint32_t pk[16];
+        {
+          const uint32_t ew[16] = {ec[0].x, ec[0].y, ec[0].z, ec[0].w, ec[1].x, ec[1].y, ec[1].z, ec[1].w,
+                                   ec[2].x, ec[2].y, ec[2].z, ec[2].w, ec[3].x, ec[3].y, ec[3].z, ec[3].w};
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
-        const bool full = col0 + 32 <= G.N;
-        if (E) {
-          const __nv_bfloat16* e = E + (int64_t)row * G.lde + col0;
-          if (full) {
-#pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const uint4 w = *reinterpret_cast<const uint4*>(e + 8 * j4);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                v[8 * j4 + 2 * h] += beta * bf16_bits_to_f(ww[h] & 0xFFFFu);
-                v[8 * j4 + 2 * h + 1] += beta * bf16_bits_to_f(ww[h] >> 16);
-              }
+          for (int h = 0; h < 16; ++h) {
+            float v0 = alpha * __uint_as_float(r[2 * h]), v1 = alpha * __uint_as_float(r[2 * h + 1]);
+            if (Erow) {
+              v0 += beta * bf16_bits_to_f(ew[h] & 0xFFFFu);
+              v1 += beta * bf16_bits_to_f(ew[h] >> 16);
             }
-          } else {
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < G.N) v[j] += beta * __bfloat162float(e[j]);
+            const __nv_bfloat162 p2 = __floats2bfloat162_rn(v0, v1);
+            pk[h] = *reinterpret_cast<const uint32_t*>(&p2);
           }
         }
-        __nv_bfloat16* c = C + (int64_t)row * G.ldc + col0;
-        if (!sym) {
-          if (full) {
+        // staging buffers of this parity are free once the group issued two
+        // chunks ago has been read by the TMA unit
+        if (lane == 0) bulk_wait_read1();
+        __syncwarp();
+        const uint32_t dbuf = wbuf + par * 2u * kOutTileBytes, mbuf = dbuf + kOutTileBytes;
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              uint32_t w[4];
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * j4 + 2 * h], v[8 * j4 + 2 * h + 1]);
-                w[h] = *reinterpret_cast<const uint32_t*>(&p);
-              }
-              *reinterpret_cast<uint4*>(c + 8 * j4) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          } else {
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < G.N) c[j] = __float2bfloat16_rn(v[j]);
-          }
-        } else {
-          // direct: col >= row ; mirror: col > row
-#pragma unroll 4
-          for (int j = 0; j < 32; ++j) {
-            const int col = col0 + j;
-            if (col >= G.N) break;
-            if (col >= row) {
-              const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
-              c[j] = h;
-              if (col > row) C[(int64_t)col * G.ldc + row] = h;
-            }
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(dbuf + swz64(lane, 16 * c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        const bool diag = sym && col0 == r0;
+        const bool mirror = sym && col0 > r0;
+        if (diag) {
+          __syncwarp();
+          // lower part of the diagonal block <- its upper part (element (j, lane) of row j)
+          for (int j = 0; j < lane; ++j) {
+            const uint16_t h = ld_shared_u16(dbuf + swz64(j, 2 * lane));
+            st_shared_u16(dbuf + swz64(lane, 2 * j), h);
           }
         }
+        if (mirror) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            st_shared_u16(mbuf + swz64(j, 2 * lane), (uint16_t)(pk[j >> 1] >> (16 * (j & 1))));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(mC, dbuf, col0, r0, ti.b);
+          if (mirror) tma_store_3d(mC, mbuf, r0, col0, ti.b);
+          bulk_commit();
+        }
+        par ^= 1u;
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
       if (acc == 1) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -428,7 +488,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t ld_elems,
-               uint64_t batch_elems, uint32_t box0, uint32_t box1) {
+               uint64_t batch_elems, uint32_t box0, uint32_t box1,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = get_encode();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
@@ -436,7 +497,7 @@ bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uin
   const cuuint32_t box[3] = {box0, box1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -466,13 +527,15 @@ bool tc_encode_maps(const GemmLaunch& L, void* maps_out) {
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_out);
   for (int g = 0; g < L.num_groups; ++g) {
     const GemmGroup& G = L.g[g];
-    if (!encode_3d(&maps[2 * g], G.A, G.K, G.M, G.count, G.lda, G.sa, TBK, TBM)) return false;
+    if (!encode_3d(&maps[3 * g], G.A, G.K, G.M, G.count, G.lda, G.sa, TBK, TBM)) return false;
     bool ok;
     if (G.kind == GK_UPD)
-      ok = encode_3d(&maps[2 * g + 1], G.B, G.N, G.K, G.count, G.ldb, G.sb, 64, TBK);
+      ok = encode_3d(&maps[3 * g + 1], G.B, G.N, G.K, G.count, G.ldb, G.sb, 64, TBK);
     else
-      ok = encode_3d(&maps[2 * g + 1], G.B, G.K, G.N, G.count, G.ldb, G.sb, TBK, TBN);
+      ok = encode_3d(&maps[3 * g + 1], G.B, G.K, G.N, G.count, G.ldb, G.sb, TBK, TBN);
     if (!ok) return false;
+    if (!encode_3d(&maps[3 * g + 2], G.C, G.N, G.M, G.count, G.ldc, G.sc, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return false;
   }
   return true;
 }
@@ -486,7 +549,7 @@ cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, c
   });
   if (attr_err != cudaSuccess) return attr_err;
   TcParams* P = new TcParams;
-  std::memcpy(P->maps, maps, sizeof(CUtensorMap) * 2 * L.num_groups);
+  std::memcpy(P->maps, maps, sizeof(CUtensorMap) * 3 * L.num_groups);
   P->L = L;
   const int grid = std::min(num_sms, L.total_tiles);
   k_gemm_tc<<<grid, kThreads, kSmemBytes, st>>>(*P);

@@ -46,7 +46,7 @@ struct GemmLaunch {
 cudaError_t launch_gemm_simt(const GemmLaunch& L, cudaStream_t st);
 
 // tcgen05 grouped GEMM (bf16 operands, fp32 accumulation in TMEM, TMA loads).
-// `maps` holds two CUtensorMap (128 B each) per group: operand A, operand B.
+// `maps` holds three CUtensorMap (128 B each) per group: operand A, operand B, output C.
 struct TcLaunch;
 cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, cudaStream_t st);
 bool tc_encode_maps(const GemmLaunch& L, void* maps_out);  // host: builds the tensor maps
