@@ -24,6 +24,62 @@ __device__ __forceinline__ void st_from_f32(void* p, int64_t i, int dt, float v)
 }
 __host__ __device__ __forceinline__ int dt_bytes(int dt) { return dt == kBF16 ? 2 : 4; }
 
+// 8 consecutive elements p[i .. i+7] as floats; i a multiple of 8 and the
+// array 16-byte aligned (one 16-byte load for bf16, two for fp32).
+__device__ __forceinline__ void ld8(const void* p, int64_t i, int dt, float (&v)[8]) {
+  if (dt == kBF16) {
+    const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + i);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      v[2 * h] = __uint_as_float(ww[h] << 16);
+      v[2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i);
+    const float4 b = *(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+__device__ __forceinline__ void st8(void* p, int64_t i, int dt, const float (&v)[8]) {
+  if (dt == kBF16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * h], v[2 * h + 1]);
+      w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + i) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    float4* q = reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + i);
+    q[0] = make_float4(v[0], v[1], v[2], v[3]);
+    q[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+// Masked variants: only elements k < cnt (cnt <= 8) are touched; others read 0.
+__device__ __forceinline__ void ld8m(const void* p, int64_t i, int dt, int cnt, float (&v)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = k < cnt ? ld_as_f32(p, i + k, dt) : 0.f;
+}
+__device__ __forceinline__ void st8m(void* p, int64_t i, int dt, int cnt, const float (&v)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (k < cnt) st_from_f32(p, i + k, dt, v[k]);
+}
+// Vector or masked access of the 8-group starting at column j of a row of
+// length n (row start index `row_off`); vec: rows are 16-byte aligned.
+__device__ __forceinline__ void ld8r(const void* p, int64_t row_off, int64_t j, int64_t n, bool vec, int dt,
+                                     float (&v)[8]) {
+  if (vec && j + 8 <= n) ld8(p, row_off + j, dt, v);
+  else ld8m(p, row_off + j, dt, (int)(n - j < 8 ? (n - j > 0 ? n - j : 0) : 8), v);
+}
+__device__ __forceinline__ void st8r(void* p, int64_t row_off, int64_t j, int64_t n, bool vec, int dt,
+                                     const float (&v)[8]) {
+  if (vec && j + 8 <= n) st8(p, row_off + j, dt, v);
+  else st8m(p, row_off + j, dt, (int)(n - j < 8 ? (n - j > 0 ? n - j : 0) : 8), v);
+}
+
 // ---------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

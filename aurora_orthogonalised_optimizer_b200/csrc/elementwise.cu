@@ -15,13 +15,15 @@
 namespace am {
 
 constexpr int kTile = 64;       // element-wise tile edge
-constexpr int kEwThreads = 256; // 64 columns x 4 row lanes
+constexpr int kEwThreads = 256; // 8 column groups of 8 elements x 32 row lanes
 
 // ============================================================================
 // prologue: m <- m + (1-mu)(g-m); u = Nesterov ? g + mu(m-g) : m; write u in
 // the X orientation (transposed through shared memory for tall matrices);
 // per-block partials of |u|^2 and |W|^2.
 // mode 0: optimizer step (uses G, M, W);  mode 1: u = G (input staging).
+// A block owns a 64 x 64 tile; thread t handles the 8-element groups
+// (row t/8 + 32k, columns 8 (t%8) .. +7), k = 0, 1, with 16-byte accesses.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, double* partials) {
@@ -32,37 +34,64 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
   const int b = blockIdx.x - t.blk_prefix[mi];
   const int64_t tiles_c = (d.n + kTile - 1) / kTile;
   const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+  const bool vec = (d.n & 7) == 0;
+  const bool xvec = (d.ldl & 7) == 0;
   float su2 = 0.f, sw2 = 0.f;
-  const int64_t j = c0 + tx;
-#pragma unroll 4
-  for (int rr = ty; rr < kTile; rr += 4) {
+  const int64_t j = c0 + 8 * cg;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int rr = rg + 32 * k;
     const int64_t i = r0 + rr;
-    float u = 0.f;
+    float u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (i < d.m && j < d.n) {
-      const int64_t e = i * d.n + j;
-      const float g = ld_as_f32(d.G, e, t.grad_dtype);
+      const int64_t ro = i * d.n;
+      float g[8];
+      ld8r(d.G, ro, j, d.n, vec, t.grad_dtype, g);
       if (mode == 0) {
-        const float m0 = d.M[e];
-        const float m1 = m0 + (1.f - mu) * (g - m0);
-        d.M[e] = m1;
-        u = nesterov ? g + mu * (m1 - g) : m1;
-        if (want_w2) { const float w = ld_as_f32(d.W, e, t.param_dtype); sw2 += w * w; }
+        float m[8];
+        ld8r(d.M, ro, j, d.n, vec, kF32, m);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float m1 = m[e] + (1.f - mu) * (g[e] - m[e]);
+          m[e] = m1;
+          u[e] = nesterov ? g[e] + mu * (m1 - g[e]) : m1;
+        }
+        st8r(d.M, ro, j, d.n, vec, kF32, m);
+        if (want_w2) {
+          float w[8];
+          ld8r(d.W, ro, j, d.n, vec, t.param_dtype, w);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sw2 += w[e] * w[e];
+        }
       } else {
-        u = g;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u[e] = g[e];
       }
-      su2 += u * u;
-      if (!d.tall) st_from_f32(d.uX, i * d.ldl + j, t.ns_dtype, u);
+      if (j + 8 > d.n)
+        for (int e = (int)(d.n - j); e < 8; ++e) u[e] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) su2 += u[e] * u[e];
+      if (!d.tall) st8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
     }
-    tile[rr][tx] = u;
+    if (d.tall) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tile[rr][8 * cg + e] = u[e];
+    }
   }
   if (d.tall) {
     __syncthreads();
-    // X row = original column c0 + rr, X column = original row r0 + tx
-#pragma unroll 4
-    for (int rr = ty; rr < kTile; rr += 4) {
-      const int64_t xi = c0 + rr, xj = r0 + tx;
-      if (xi < d.n && xj < d.m) st_from_f32(d.uX, xi * d.ldl + xj, t.ns_dtype, tile[tx][rr]);
+    // X row = original column c0 + xr; X columns = original rows r0 + 8 cg ..
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int xr = rg + 32 * k;
+      const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
+      if (xi < d.n && xj < d.m) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = tile[8 * cg + e][xr];
+        st8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, v);
+      }
     }
   }
   const double a = block_sum((double)su2, red);
@@ -94,37 +123,49 @@ __global__ void k_finalize_sums(const MatTable t, const double* partials, int nq
 //   mode 0 (D init):  D_j = 1 / max(sqrt(sum), pp_eps)              ["源码实现"]
 //   mode 1 (D update): row_sq = max(sum, pp_eps^2);
 //                      D_j *= (target / row_sq)^beta, target = s / l
+// A block owns 64 columns: 8 column groups of 8 x 32 row lanes, 16-byte loads.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
-  __shared__ float part[4][kTile];
+  __shared__ float part[32][kTile + 1];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
-  const int64_t j = (int64_t)b * kTile + tx;
+  const int cg = threadIdx.x & 7, rl = threadIdx.x >> 3;
+  const int64_t j = (int64_t)b * kTile + 8 * cg;
   const void* X = mode == 0 ? d.uX : d.UX;
-  float acc = 0.f;
-  if (j < d.l)
-    for (int64_t i = ty; i < d.s; i += 4) {
-      const float x = ld_as_f32(X, i * d.ldl + j, t.ns_dtype);
-      acc += x * x;
+  const bool vec = (d.ldl & 7) == 0;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (j < d.l) {
+#pragma unroll 4
+    for (int64_t i = rl; i < d.s; i += 32) {
+      float x[8];
+      ld8r(X, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += x[e] * x[e];
     }
-  part[ty][tx] = acc;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[rl][8 * cg + e] = acc[e];
   __syncthreads();
-  if (ty == 0 && j < d.l) {
-    const float sum = ((part[0][tx] + part[1][tx]) + part[2][tx]) + part[3][tx];
-    if (mode == 0) {
-      d.D[j] = 1.f / fmaxf(sqrtf(sum), pp_eps);
-    } else {
-      const float row_sq = fmaxf(sum, pp_eps * pp_eps);
-      const float target = (float)d.s / (float)d.l;
-      d.D[j] = d.D[j] * powf(target / row_sq, beta);
+  if (threadIdx.x < kTile) {
+    const int64_t jj = (int64_t)b * kTile + threadIdx.x;
+    if (jj < d.l) {
+      float sum = 0.f;
+      for (int r = 0; r < 32; ++r) sum += part[r][threadIdx.x];
+      if (mode == 0) {
+        d.D[jj] = 1.f / fmaxf(sqrtf(sum), pp_eps);
+      } else {
+        const float row_sq = fmaxf(sum, pp_eps * pp_eps);
+        const float target = (float)d.s / (float)d.l;
+        d.D[jj] = d.D[jj] * powf(target / row_sq, beta);
+      }
     }
   }
 }
 
 // X0 = uX * diag(D) in the NS dtype, with per-block partials of |X0|^2.
+// 64 x 64 tiles of the X orientation, 8-element groups.
 __global__ void __launch_bounds__(kEwThreads)
 k_scale_cols(const MatTable t, double* partials) {
   __shared__ double red[32];
@@ -133,17 +174,25 @@ k_scale_cols(const MatTable t, double* partials) {
   const int b = blockIdx.x - t.blk_prefix[mi];
   const int64_t tiles_c = (d.l + kTile - 1) / kTile;
   const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
-  const int64_t j = c0 + tx;
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+  const int64_t j = c0 + 8 * cg;
+  const bool vec = (d.ldl & 7) == 0;
   float s2 = 0.f;
   if (j < d.l) {
-    const float dj = d.D[j];
-    for (int rr = ty; rr < kTile; rr += 4) {
-      const int64_t i = r0 + rr;
+    float dj[8];
+    ld8r(d.D, 0, j, d.l, true, kF32, dj);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t i = r0 + rg + 32 * k;
       if (i < d.s) {
-        const float x = ld_as_f32(d.uX, i * d.ldl + j, t.ns_dtype) * dj;
-        s2 += x * x;
-        st_from_f32(d.X0, i * d.ldl + j, t.ns_dtype, x);
+        float x[8];
+        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[e] *= dj[e];
+          s2 += x[e] * x[e];
+        }
+        st8r(d.X0, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
       }
     }
   }
@@ -212,36 +261,61 @@ __global__ void k_scalars(const MatTable t, int op, int src_slot, float ns_eps, 
 // Power iteration ("组合优化栈": scale_to_unit_operator_norm, 5 iterations).
 // On the X orientation Q (s x l):
 //   flag 0 (row dot):  out_i = sum_j Q_ij x_j   (x length l, out length s)
+//                      one warp per row, 8-element groups per lane
 //   flag 1 (col dot):  out_j = sum_i Q_ij y_i   (y length s, out length l)
-// `dir` selects vec0 -> vec1 (0) or vec1 -> vec0 (1).
+//                      64 columns per block, 8 groups x 32 row lanes
+// `dir` selects vec0 -> vec1 (0) or vec1 -> vec0 (1).  The vectors are
+// 16-byte aligned with length padded to a multiple of 64.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_matvec(const MatTable t, int dir) {
-  __shared__ float part[4][kTile];
+  __shared__ float part[32][kTile + 1];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
   const float* in = dir == 0 ? d.vec0 : d.vec1;
   float* out = dir == 0 ? d.vec1 : d.vec0;
+  const bool vec = (d.ldl & 7) == 0;
   if (d.flag == 0) {
-    // 8 warps, one row each
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t i = (int64_t)b * 8 + w;
     if (i < d.s) {
       float acc = 0.f;
-      for (int64_t j = lane; j < d.l; j += 32) acc += ld_as_f32(d.uX, i * d.ldl + j, t.ns_dtype) * in[j];
+      for (int64_t j = 8 * lane; j < d.l; j += 256) {
+        float x[8], v[8];
+        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+        ld8r(in, 0, j, d.l, true, kF32, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc += x[e] * v[e];
+      }
       acc = warp_sum(acc);
       if (lane == 0) out[i] = acc;
     }
   } else {
-    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
-    const int64_t j = (int64_t)b * kTile + tx;
-    float acc = 0.f;
-    if (j < d.l)
-      for (int64_t i = ty; i < d.s; i += 4) acc += ld_as_f32(d.uX, i * d.ldl + j, t.ns_dtype) * in[i];
-    part[ty][tx] = acc;
+    const int cg = threadIdx.x & 7, rl = threadIdx.x >> 3;
+    const int64_t j = (int64_t)b * kTile + 8 * cg;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (j < d.l) {
+#pragma unroll 4
+      for (int64_t i = rl; i < d.s; i += 32) {
+        float x[8];
+        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+        const float y = in[i];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += x[e] * y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[rl][8 * cg + e] = acc[e];
     __syncthreads();
-    if (ty == 0 && j < d.l) out[j] = ((part[0][tx] + part[1][tx]) + part[2][tx]) + part[3][tx];
+    if (threadIdx.x < kTile) {
+      const int64_t jj = (int64_t)b * kTile + threadIdx.x;
+      if (jj < d.l) {
+        float sum = 0.f;
+        for (int r = 0; r < 32; ++r) sum += part[r][threadIdx.x];
+        out[jj] = sum;
+      }
+    }
   }
 }
 
@@ -283,19 +357,26 @@ k_dots(const MatTable t, double* partials) {
   const int b = blockIdx.x - t.blk_prefix[mi];
   const int64_t tiles_c = (d.l + kTile - 1) / kTile;
   const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
-  const int64_t j = c0 + tx;
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+  const int64_t j = c0 + 8 * cg;
+  const bool vec = (d.ldl & 7) == 0;
   float a = 0.f, c = 0.f;
-  if (j < d.l)
-    for (int rr = ty; rr < kTile; rr += 4) {
-      const int64_t i = r0 + rr;
+  if (j < d.l) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t i = r0 + rg + 32 * k;
       if (i < d.s) {
-        const float U = ld_as_f32(d.UX, i * d.ldl + j, t.ns_dtype);
-        const float u = ld_as_f32(d.uX, i * d.ldl + j, t.ns_dtype);
-        a += U * U;
-        c += U * u;
+        float U[8], u[8];
+        ld8r(d.UX, i * d.ldl, j, d.l, vec, t.ns_dtype, U);
+        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          a += U[e] * U[e];
+          c += U[e] * u[e];
+        }
       }
     }
+  }
   const double A = block_sum((double)a, red);
   const double C = block_sum((double)c, red);
   if (threadIdx.x == 0) {
@@ -308,6 +389,7 @@ k_dots(const MatTable t, double* partials) {
 // Fused epilogue, original orientation: V = cU U + cu u (U, u read from the
 // X orientation, transposed through shared memory for tall matrices);
 // optional fp32 V output; optional W <- W - lr V in the param dtype.
+// 64 x 64 tiles, 8-element groups with 16-byte accesses.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
@@ -318,45 +400,69 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
   const int b = blockIdx.x - t.blk_prefix[mi];
   const int64_t tiles_c = (d.n + kTile - 1) / kTile;
   const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
   const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
   const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
-  const bool need_u = cu != 0.f;
+  const bool need_U = cU != 0.f, need_u = cu != 0.f;
+  const bool vec = (d.n & 7) == 0;
+  const bool xvec = (d.ldl & 7) == 0;
   if (d.tall) {
-    // X tile rows = original columns c0.., X tile cols = original rows r0..
-    for (int rr = ty; rr < kTile; rr += 4) {
-      const int64_t xi = c0 + rr, xj = r0 + tx;
-      const bool in = xi < d.n && xj < d.m;
-      tU[rr][tx] = in && cU != 0.f ? ld_as_f32(d.UX, xi * d.ldl + xj, t.ns_dtype) : 0.f;
-      tu[rr][tx] = in && need_u ? ld_as_f32(d.uX, xi * d.ldl + xj, t.ns_dtype) : 0.f;
+    // X tile rows = original columns c0 + xr, X tile columns = original rows r0 + 8 cg ..
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int xr = rg + 32 * k;
+      const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
+      float U[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (xi < d.n && xj < d.m) {
+        if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, U);
+        if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, u);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        tU[xr][8 * cg + e] = U[e];
+        tu[xr][8 * cg + e] = u[e];
+      }
     }
     __syncthreads();
   }
-  const int64_t j = c0 + tx;
-  for (int rr = ty; rr < kTile; rr += 4) {
+  const int64_t j = c0 + 8 * cg;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int rr = rg + 32 * k;
     const int64_t i = r0 + rr;
     if (i >= d.m || j >= d.n) continue;
-    float U, u;
+    float U[8], u[8];
     if (d.tall) {
-      U = tU[tx][rr];
-      u = tu[tx][rr];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        U[e] = tU[8 * cg + e][rr];
+        u[e] = tu[8 * cg + e][rr];
+      }
     } else {
-      U = cU != 0.f ? ld_as_f32(d.UX, i * d.ldl + j, t.ns_dtype) : 0.f;
-      u = need_u ? ld_as_f32(d.uX, i * d.ldl + j, t.ns_dtype) : 0.f;
+      if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U);
+      else for (int e = 0; e < 8; ++e) U[e] = 0.f;
+      if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
+      else for (int e = 0; e < 8; ++e) u[e] = 0.f;
     }
-    const float v = cU * U + cu * u;
-    const int64_t e = i * d.n + j;
-    if (d.V) d.V[e] = v;
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = cU * U[e] + cu * u[e];
+    const int64_t ro = i * d.n;
+    if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v);
     if (update_w) {
-      const float w = ld_as_f32(d.W, e, t.param_dtype);
-      st_from_f32(d.W, e, t.param_dtype, w - lr * v);
+      float w[8];
+      ld8r(d.W, ro, j, d.n, vec, t.param_dtype, w);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] -= lr * v[e];
+      st8r(d.W, ro, j, d.n, vec, t.param_dtype, w);
     }
   }
 }
 
 // ============================================================================
 // u/w floor on caller-provided fp32 updates (entry point uw_floor_apply):
-// partial |W|^2 and |V|^2 over the original orientation, then V *= coef.
+// partial |W|^2 and |V|^2 over the flat original layout (4096 elements per
+// block, 16-byte accesses), then V *= coef.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_sumsq_wv(const MatTable t, double* partials) {
@@ -366,12 +472,19 @@ k_sumsq_wv(const MatTable t, double* partials) {
   const int b = blockIdx.x - t.blk_prefix[mi];
   const int64_t total = d.m * d.n;
   float sw = 0.f, sv = 0.f;
-  for (int64_t e = (int64_t)b * 4096 + threadIdx.x; e < total && e < (int64_t)(b + 1) * 4096;
-       e += blockDim.x) {
-    const float w = ld_as_f32(d.W, e, t.param_dtype);
-    const float v = d.V[e];
-    sw += w * w;
-    sv += v * v;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int64_t e0 = (int64_t)b * 4096 + 8 * (threadIdx.x + 256 * k);
+    if (e0 < total) {
+      float w[8], v[8];
+      ld8r(d.W, 0, e0, total, true, t.param_dtype, w);
+      ld8r(d.V, 0, e0, total, true, kF32, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sw += w[e] * w[e];
+        sv += v[e] * v[e];
+      }
+    }
   }
   const double W2 = block_sum((double)sw, red);
   const double V2 = block_sum((double)sv, red);
@@ -389,9 +502,17 @@ k_scale_v(const MatTable t, const double* scal) {
   const float c = (float)scal[d.idx * S_COUNT + S_COEF_U];
   if (c == 1.f) return;
   const int64_t total = d.m * d.n;
-  for (int64_t e = (int64_t)b * 4096 + threadIdx.x; e < total && e < (int64_t)(b + 1) * 4096;
-       e += blockDim.x)
-    d.V[e] *= c;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int64_t e0 = (int64_t)b * 4096 + 8 * (threadIdx.x + 256 * k);
+    if (e0 < total) {
+      float v[8];
+      ld8r(d.V, 0, e0, total, true, kF32, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] *= c;
+      st8r(d.V, 0, e0, total, true, kF32, v);
+    }
+  }
 }
 
 // rho (double, scalar block) -> bucket-ordered float slot for the GEMMs.

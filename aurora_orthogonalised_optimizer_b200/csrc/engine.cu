@@ -28,6 +28,7 @@ constexpr size_t kAlign = 1024;
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
+inline int64_t round64(int64_t x) { return (x + 63) / 64 * 64; }
 
 struct MatPlan {
   int64_t m, n, s, l;
@@ -93,9 +94,10 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
     b.off_Q = off;  off = align_up(off + xbytes);
     b.off_A = off;  off = align_up(off + abytes);
     b.off_B = off;  off = align_up(off + abytes);
-    b.off_D = off;  off = align_up(off + cnt * (size_t)b.l * 4);
-    b.off_v0 = off; off = align_up(off + cnt * (size_t)b.l * 4);
-    b.off_v1 = off; off = align_up(off + cnt * (size_t)b.l * 4);
+    const size_t vbytes = cnt * (size_t)round64(b.l) * 4;   // per-matrix vectors, 256-byte aligned
+    b.off_D = off;  off = align_up(off + vbytes);
+    b.off_v0 = off; off = align_up(off + vbytes);
+    b.off_v1 = off; off = align_up(off + vbytes);
     b.off_rho = off; off = align_up(off + cnt * 4);
   }
   p.off_scal = off;
@@ -241,9 +243,10 @@ MatDesc make_desc(const Ctx& c, int i) {
   const bool odd = (c.cfg->ns_steps & 1) != 0;
   d.UX = c.ws + (odd ? b.off_P : b.off_Q) + xo;
   d.X0 = c.ws + b.off_Q + xo;
-  d.D = wsp<float>(c, b.off_D) + (size_t)mp.bidx * b.l;
-  d.vec0 = wsp<float>(c, b.off_v0) + (size_t)mp.bidx * b.l;
-  d.vec1 = wsp<float>(c, b.off_v1) + (size_t)mp.bidx * b.l;
+  const size_t vo = (size_t)mp.bidx * (size_t)round64(b.l);
+  d.D = wsp<float>(c, b.off_D) + vo;
+  d.vec0 = wsp<float>(c, b.off_v0) + vo;
+  d.vec1 = wsp<float>(c, b.off_v1) + vo;
   d.rho_slot = wsp<float>(c, b.off_rho) + mp.bidx;
   d.m = mp.m; d.n = mp.n; d.s = mp.s; d.l = mp.l; d.ldl = b.ldl;
   d.tall = mp.tall;
