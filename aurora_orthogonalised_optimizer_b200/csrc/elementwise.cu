@@ -16,19 +16,33 @@ namespace am {
 
 constexpr int kTile = 64;       // element-wise tile edge
 constexpr int kEwThreads = 256; // 8 column groups of 8 elements x 32 row lanes
+constexpr int kWarps = kEwThreads / 32;
+
+// Warp-level partial sums (no block barrier): lane 0 of each warp writes
+// its warp's sums to partials[((slot) * kWarps + warp) * nq + q].
+__device__ __forceinline__ void warp_partials(double* partials, int64_t slot, int nq, float a, float b) {
+  const double A = warp_sum((double)a);
+  const double B = nq > 1 ? warp_sum((double)b) : 0.0;
+  if ((threadIdx.x & 31) == 0) {
+    double* p = partials + (slot * kWarps + (threadIdx.x >> 5)) * nq;
+    p[0] = A;
+    if (nq > 1) p[1] = B;
+  }
+}
 
 // ============================================================================
 // prologue: m <- m + (1-mu)(g-m); u = Nesterov ? g + mu(m-g) : m; write u in
 // the X orientation (transposed through shared memory for tall matrices);
-// per-block partials of |u|^2 and |W|^2.
+// per-warp partials of |u|^2 and |W|^2.
 // mode 0: optimizer step (uses G, M, W);  mode 1: u = G (input staging).
 // A block owns a 64 x 64 tile; thread t handles the 8-element groups
 // (row t/8 + 32k, columns 8 (t%8) .. +7), k = 0, 1, with 16-byte accesses.
+// All loads are issued before any store (the buffers may alias as far as the
+// compiler knows).
 // ============================================================================
-__global__ void __launch_bounds__(kEwThreads)
+__global__ void __launch_bounds__(kEwThreads, 4)
 k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, double* partials) {
   __shared__ float tile[kTile][kTile + 1];
-  __shared__ double red[32];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
@@ -37,49 +51,51 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
   const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
   const bool vec = (d.n & 7) == 0;
   const bool xvec = (d.ldl & 7) == 0;
-  float su2 = 0.f, sw2 = 0.f;
   const int64_t j = c0 + 8 * cg;
+  const bool in0 = r0 + rg < d.m && j < d.n, in1 = r0 + rg + 32 < d.m && j < d.n;
+  const int64_t ro0 = (r0 + rg) * d.n, ro1 = (r0 + rg + 32) * d.n;
+  float g0[8], g1[8], m0[8], m1[8], w0[8], w1[8];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int rr = rg + 32 * k;
-    const int64_t i = r0 + rr;
-    float u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (i < d.m && j < d.n) {
-      const int64_t ro = i * d.n;
-      float g[8];
-      ld8r(d.G, ro, j, d.n, vec, t.grad_dtype, g);
-      if (mode == 0) {
-        float m[8];
-        ld8r(d.M, ro, j, d.n, vec, kF32, m);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float m1 = m[e] + (1.f - mu) * (g[e] - m[e]);
-          m[e] = m1;
-          u[e] = nesterov ? g[e] + mu * (m1 - g[e]) : m1;
-        }
-        st8r(d.M, ro, j, d.n, vec, kF32, m);
-        if (want_w2) {
-          float w[8];
-          ld8r(d.W, ro, j, d.n, vec, t.param_dtype, w);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) sw2 += w[e] * w[e];
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) u[e] = g[e];
-      }
-      if (j + 8 > d.n)
-        for (int e = (int)(d.n - j); e < 8; ++e) u[e] = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) su2 += u[e] * u[e];
-      if (!d.tall) st8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
-    }
-    if (d.tall) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) tile[rr][8 * cg + e] = u[e];
+  for (int e = 0; e < 8; ++e) g0[e] = g1[e] = m0[e] = m1[e] = w0[e] = w1[e] = 0.f;
+  if (in0) ld8r(d.G, ro0, j, d.n, vec, t.grad_dtype, g0);
+  if (in1) ld8r(d.G, ro1, j, d.n, vec, t.grad_dtype, g1);
+  if (mode == 0) {
+    if (in0) ld8r(d.M, ro0, j, d.n, vec, kF32, m0);
+    if (in1) ld8r(d.M, ro1, j, d.n, vec, kF32, m1);
+    if (want_w2) {
+      if (in0) ld8r(d.W, ro0, j, d.n, vec, t.param_dtype, w0);
+      if (in1) ld8r(d.W, ro1, j, d.n, vec, t.param_dtype, w1);
     }
   }
-  if (d.tall) {
+  float su2 = 0.f, sw2 = 0.f;
+  float u0[8], u1[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if (mode == 0) {
+      m0[e] = m0[e] + (1.f - mu) * (g0[e] - m0[e]);
+      m1[e] = m1[e] + (1.f - mu) * (g1[e] - m1[e]);
+      u0[e] = nesterov ? g0[e] + mu * (m0[e] - g0[e]) : m0[e];
+      u1[e] = nesterov ? g1[e] + mu * (m1[e] - g1[e]) : m1[e];
+    } else {
+      u0[e] = g0[e];
+      u1[e] = g1[e];
+    }
+    su2 += u0[e] * u0[e] + u1[e] * u1[e];
+    sw2 += w0[e] * w0[e] + w1[e] * w1[e];
+  }
+  if (mode == 0) {
+    if (in0) st8r(d.M, ro0, j, d.n, vec, kF32, m0);
+    if (in1) st8r(d.M, ro1, j, d.n, vec, kF32, m1);
+  }
+  if (!d.tall) {
+    if (in0) st8r(d.uX, (r0 + rg) * d.ldl, j, d.n, xvec, t.ns_dtype, u0);
+    if (in1) st8r(d.uX, (r0 + rg + 32) * d.ldl, j, d.n, xvec, t.ns_dtype, u1);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      tile[rg][8 * cg + e] = u0[e];
+      tile[rg + 32][8 * cg + e] = u1[e];
+    }
     __syncthreads();
     // X row = original column c0 + xr; X columns = original rows r0 + 8 cg ..
 #pragma unroll
@@ -94,16 +110,11 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
       }
     }
   }
-  const double a = block_sum((double)su2, red);
-  const double w = block_sum((double)sw2, red);
-  if (threadIdx.x == 0) {
-    partials[(int64_t)(d.part + b) * 2 + 0] = a;
-    partials[(int64_t)(d.part + b) * 2 + 1] = w;
-  }
+  warp_partials(partials, d.part + b, 2, su2, sw2);
 }
 
-// Sum the per-block partials of each matrix into its scalar block.
-// partials are laid out [slot q of nq] per block.  dst_slot[q] < 0 skips q.
+// Sum the per-warp partials of each matrix into its scalar block.  Layout:
+// partials[((part + block) * 8 + warp) * nq + q]; slot < 0 skips q.
 __global__ void k_finalize_sums(const MatTable t, const double* partials, int nq, int slot0,
                                 int slot1, double* scal) {
   __shared__ double red[32];
@@ -111,7 +122,8 @@ __global__ void k_finalize_sums(const MatTable t, const double* partials, int nq
   for (int q = 0; q < nq; ++q) {
     const int slot = q == 0 ? slot0 : slot1;
     double s = 0.0;
-    for (int b = threadIdx.x; b < d.nblk; b += blockDim.x) s += partials[(int64_t)(d.part + b) * nq + q];
+    const int64_t n = (int64_t)d.nblk * kWarps;
+    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) s += partials[((int64_t)d.part * kWarps + k) * nq + q];
     s = block_sum(s, red);
     if (threadIdx.x == 0 && slot >= 0) scal[d.idx * S_COUNT + slot] = s;
   }
@@ -164,11 +176,10 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
   }
 }
 
-// X0 = uX * diag(D) in the NS dtype, with per-block partials of |X0|^2.
+// X0 = uX * diag(D) in the NS dtype, with per-warp partials of |X0|^2.
 // 64 x 64 tiles of the X orientation, 8-element groups.
 __global__ void __launch_bounds__(kEwThreads)
 k_scale_cols(const MatTable t, double* partials) {
-  __shared__ double red[32];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
@@ -179,25 +190,22 @@ k_scale_cols(const MatTable t, double* partials) {
   const bool vec = (d.ldl & 7) == 0;
   float s2 = 0.f;
   if (j < d.l) {
-    float dj[8];
+    const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
+    const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
+    float dj[8], x0[8], x1[8];
     ld8r(d.D, 0, j, d.l, true, kF32, dj);
+    if (in0) ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, x0);
+    if (in1) ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, x1);
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t i = r0 + rg + 32 * k;
-      if (i < d.s) {
-        float x[8];
-        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] *= dj[e];
-          s2 += x[e] * x[e];
-        }
-        st8r(d.X0, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
-      }
+    for (int e = 0; e < 8; ++e) {
+      x0[e] = in0 ? x0[e] * dj[e] : 0.f;
+      x1[e] = in1 ? x1[e] * dj[e] : 0.f;
+      s2 += x0[e] * x0[e] + x1[e] * x1[e];
     }
+    if (in0) st8r(d.X0, ro0, j, d.l, vec, t.ns_dtype, x0);
+    if (in1) st8r(d.X0, ro1, j, d.l, vec, t.ns_dtype, x1);
   }
-  const double a = block_sum((double)s2, red);
-  if (threadIdx.x == 0) partials[d.part + b] = a;
+  warp_partials(partials, d.part + b, 1, s2, 0.f);
 }
 
 // Per-matrix scalar algebra (one thread per matrix).
@@ -347,11 +355,10 @@ __global__ void k_vecop(const MatTable t, int which, int mode, int len_is_s_when
 }
 
 // ============================================================================
-// <U,U> and <U,u> over the X orientation, per-block partials (2 per block).
+// <U,U> and <U,u> over the X orientation, per-warp partials (2 per warp).
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_dots(const MatTable t, double* partials) {
-  __shared__ double red[32];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
@@ -362,27 +369,20 @@ k_dots(const MatTable t, double* partials) {
   const bool vec = (d.ldl & 7) == 0;
   float a = 0.f, c = 0.f;
   if (j < d.l) {
+    const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
+    const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
+    float U0[8], u0[8], U1[8], u1[8];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t i = r0 + rg + 32 * k;
-      if (i < d.s) {
-        float U[8], u[8];
-        ld8r(d.UX, i * d.ldl, j, d.l, vec, t.ns_dtype, U);
-        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, u);
+    for (int e = 0; e < 8; ++e) U0[e] = u0[e] = U1[e] = u1[e] = 0.f;
+    if (in0) { ld8r(d.UX, ro0, j, d.l, vec, t.ns_dtype, U0); ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, u0); }
+    if (in1) { ld8r(d.UX, ro1, j, d.l, vec, t.ns_dtype, U1); ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, u1); }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          a += U[e] * U[e];
-          c += U[e] * u[e];
-        }
-      }
+    for (int e = 0; e < 8; ++e) {
+      a += U0[e] * U0[e] + U1[e] * U1[e];
+      c += U0[e] * u0[e] + U1[e] * u1[e];
     }
   }
-  const double A = block_sum((double)a, red);
-  const double C = block_sum((double)c, red);
-  if (threadIdx.x == 0) {
-    partials[(int64_t)(d.part + b) * 2 + 0] = A;
-    partials[(int64_t)(d.part + b) * 2 + 1] = C;
-  }
+  warp_partials(partials, d.part + b, 2, a, c);
 }
 
 // ============================================================================
@@ -391,7 +391,7 @@ k_dots(const MatTable t, double* partials) {
 // optional fp32 V output; optional W <- W - lr V in the param dtype.
 // 64 x 64 tiles, 8-element groups with 16-byte accesses.
 // ============================================================================
-__global__ void __launch_bounds__(kEwThreads)
+__global__ void __launch_bounds__(kEwThreads, 4)
 k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
   __shared__ float tU[kTile][kTile + 1];
   __shared__ float tu[kTile][kTile + 1];
@@ -426,36 +426,40 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
     __syncthreads();
   }
   const int64_t j = c0 + 8 * cg;
+  float U[2][8], u[2][8], w[2][8];
+  bool in[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int rr = rg + 32 * k;
     const int64_t i = r0 + rr;
-    if (i >= d.m || j >= d.n) continue;
-    float U[8], u[8];
+    in[k] = i < d.m && j < d.n;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) U[k][e] = u[k][e] = w[k][e] = 0.f;
+    if (!in[k]) continue;
     if (d.tall) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        U[e] = tU[8 * cg + e][rr];
-        u[e] = tu[8 * cg + e][rr];
+        U[k][e] = tU[8 * cg + e][rr];
+        u[k][e] = tu[8 * cg + e][rr];
       }
     } else {
-      if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U);
-      else for (int e = 0; e < 8; ++e) U[e] = 0.f;
-      if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
-      else for (int e = 0; e < 8; ++e) u[e] = 0.f;
+      if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U[k]);
+      if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u[k]);
     }
+    if (update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (!in[k]) continue;
+    const int64_t ro = (r0 + rg + 32 * k) * d.n;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = cU * U[e] + cu * u[e];
-    const int64_t ro = i * d.n;
-    if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v);
-    if (update_w) {
-      float w[8];
-      ld8r(d.W, ro, j, d.n, vec, t.param_dtype, w);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] -= lr * v[e];
-      st8r(d.W, ro, j, d.n, vec, t.param_dtype, w);
+    for (int e = 0; e < 8; ++e) {
+      v[e] = cU * U[k][e] + cu * u[k][e];
+      w[k][e] -= lr * v[e];
     }
+    if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v);
+    if (update_w) st8r(d.W, ro, j, d.n, vec, t.param_dtype, w[k]);
   }
 }
 
@@ -466,7 +470,6 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_sumsq_wv(const MatTable t, double* partials) {
-  __shared__ double red[32];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
@@ -486,12 +489,7 @@ k_sumsq_wv(const MatTable t, double* partials) {
       }
     }
   }
-  const double W2 = block_sum((double)sw, red);
-  const double V2 = block_sum((double)sv, red);
-  if (threadIdx.x == 0) {
-    partials[(int64_t)(d.part + b) * 2 + 0] = V2;
-    partials[(int64_t)(d.part + b) * 2 + 1] = W2;
-  }
+  warp_partials(partials, d.part + b, 2, sv, sw);
 }
 
 __global__ void __launch_bounds__(kEwThreads)

@@ -103,7 +103,7 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
   p.off_scal = off;
   off = align_up(off + (size_t)n * S_COUNT * sizeof(double));
   p.off_partials = off;
-  off = align_up(off + (size_t)part * 2 * sizeof(double));
+  off = align_up(off + (size_t)part * 8 /*warps*/ * 2 * sizeof(double));
   p.total = off;
   return p;
 }
@@ -165,6 +165,16 @@ int num_sms_current() {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cache[dev] = sms;
   return sms;
+}
+
+// Tensor-core GEMM variant: SM pairs (256 x 256 tiles) unless the
+// environment sets AURORA_MUON_TC_PAIR=0 (single-SM 128 x 256 tiles).
+bool tc_pair() {
+  static const bool pair = [] {
+    const char* e = std::getenv("AURORA_MUON_TC_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return pair;
 }
 
 // ---------------------------------------------------------------- tracing
@@ -363,9 +373,9 @@ muon_status gemm_launch(const Ctx& c, GemmLaunch& L) {
   if (L.num_groups == 0) return MUON_OK;
   if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
     alignas(64) unsigned char maps[kMaxGemmGroups * 3 * 128];
-    if (!tc_encode_maps(L, maps)) return MUON_ERR_CUDA;
+    if (!tc_encode_maps(L, tc_pair(), maps)) return MUON_ERR_CUDA;
     ProfScope ps(PC_GEMM_TC, gemm_flops(L), 0.0, c.st);
-    CK(launch_gemm_tc(L, maps, num_sms_current(), c.st));
+    CK(launch_gemm_tc(L, maps, num_sms_current(), tc_pair(), c.st));
   } else {
     ProfScope ps(PC_GEMM_SIMT, gemm_flops(L), 0.0, c.st);
     CK(launch_gemm_simt(L, c.st));
@@ -377,7 +387,7 @@ muon_status gemm_launch(const Ctx& c, GemmLaunch& L) {
 
 void add_group(const Ctx& c, GemmLaunch& L, GemmGroup g) {
   if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
-    g.tiles_per_mat = tc_tile_count(g.kind, g.M, g.N, &g.tiles_m, &g.tiles_n);
+    g.tiles_per_mat = tc_tile_count(g.kind, g.M, g.N, tc_pair(), &g.tiles_m, &g.tiles_n);
   } else {
     g.tiles_m = (int)cdiv(g.M, 64);
     g.tiles_n = (int)cdiv(g.N, 64);

@@ -4,18 +4,27 @@
 // Aurora write-up): A = X X^T, B = b A + c A^2, X' = a X + B X, with bf16
 // operands and fp32 accumulation.
 //
-// Kernel design (persistent, warp-specialised, one CTA per SM):
-//   warp 0      : TMA producer (one lane) -- 128x64 A tile + 256x64 B tile per
-//                 stage, 128-byte swizzle, 4-stage mbarrier ring
-//   warp 1      : TMEM allocator + tcgen05.mma issuer (one lane), M=128 N=256
-//                 K=16 per instruction, fp32 accumulators in TMEM, two
-//                 accumulator buffers (2 x 256 columns) so the epilogue of one
-//                 tile overlaps the main loop of the next
-//   warps 2..5  : epilogue -- tcgen05.ld 32 lanes x 32 columns per warp,
-//                 alpha*acc + beta*E, bf16 stores.  A and A^2 are symmetric:
-//                 only tiles touching the upper triangle run, and each of them
-//                 writes its upper part directly and its strictly-upper part
-//                 mirrored, so every element is written exactly once.
+// Kernel design (persistent, warp-specialised, one CTA per SM), in two
+// variants selected at compile time:
+//   * single-SM (PAIR = false): a CTA computes a 128 x 256 tile with
+//     tcgen05.mma.cta_group::1 (M = 128, N = 256); 4-stage smem ring of a
+//     128 x 64 A tile and a 256 x 64 B tile.
+//   * SM pair (PAIR = true): a cluster of two CTAs computes a 256 x 256 tile
+//     with tcgen05.mma.cta_group::2 (M = 256, N = 256) issued by the even
+//     ("leader") CTA.  Each CTA TMA-loads its own 128 rows of A and its own
+//     128 columns of B into its own shared memory (no multicast; the loads of
+//     both CTAs complete on the leader's barrier) and owns 128 rows of the
+//     fp32 accumulator in its TMEM.  6-stage ring of 2 x 16 KiB per CTA.
+//     Per FLOP this halves the B traffic of each SM.
+// Roles: warp 0 = TMA producer (one lane); warp 1 = TMEM allocator and MMA
+// issuer (one lane of the leader); warps 2..5 = epilogue.  Two 256-column
+// TMEM accumulators let the epilogue of one tile overlap the main loop of the
+// next.  Epilogue: tcgen05.ld 32 lanes x 32 columns per warp,
+// alpha*acc + beta*E, a 32 x 32 bf16 block staged in shared memory with the
+// 64-byte swizzle, TMA bulk-tensor store.  A and A^2 are symmetric: only tiles
+// touching the upper triangle run; each stores its upper blocks directly and
+// mirrored, and the diagonal block is completed from its own upper triangle,
+// so every element is written exactly once.
 // Operand majorness: Gram and square read both operands K-major; the update
 // reads X as an MN-major B operand (X is [K][N] with N contiguous).
 // Every mbarrier wait is bounded: on expiry the CTA records MUON_ERR_TIMEOUT,
@@ -25,6 +34,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include "kernels.h"
@@ -38,16 +48,26 @@ namespace {
 
 __device__ __forceinline__ void raise_status(unsigned int code) { atomicCAS(&g_device_status, 0u, code); }
 
-constexpr int TBM = 128, TBN = 256, TBK = 64, STAGES = 4;
+constexpr int TBN = 256, TBK = 64;
 constexpr int kThreads = 192;
-constexpr uint32_t kABytes = TBM * TBK * 2;           // 16 KiB
-constexpr uint32_t kBBytes = TBN * TBK * 2;           // 32 KiB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;                   // 2 accumulators x 256 fp32 columns
-constexpr uint32_t kOutTileBytes = 32 * 32 * 2;        // one staged 32x32 bf16 output block
+constexpr uint32_t kOutTileBytes = 32 * 32 * 2;       // one staged 32x32 bf16 output block
 constexpr uint32_t kOutBytes = 4 /*warps*/ * 4 /*2 parities x {direct, mirror}*/ * kOutTileBytes;
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * (size_t)kStageBytes + kOutBytes + 256;
 constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
+
+// Per-variant geometry (see the file comment).
+template <bool PAIR>
+struct Geo {
+  static constexpr int kTileM = PAIR ? 256 : 128;                       // rows of a tile
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr uint32_t kABytes = 128 * TBK * 2;                    // per CTA: 128 rows x 64
+  static constexpr uint32_t kBRows = PAIR ? 128 : 256;                  // B rows (N) per CTA
+  static constexpr uint32_t kBBytes = kBRows * TBK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * kStageBytes;    // lands on the leader's barrier
+  static constexpr size_t kSmemBytes = 1024 + kStages * (size_t)kStageBytes + kOutBytes + 256;
+};
+static_assert(Geo<true>::kSmemBytes <= 232448 && Geo<false>::kSmemBytes <= 232448, "shared memory budget");
 
 struct TcParams {
   CUtensorMap maps[3 * kMaxGemmGroups];   // per group: operand A, operand B, output C
@@ -174,6 +194,93 @@ __device__ __forceinline__ void load_e_chunk(const __nv_bfloat16* erow, int col0
   }
 }
 
+// ---------------------------------------------------------------- cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t a) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is signalled on a
+// barrier of either CTA of the pair (`mbar` is a shared::cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t mbar, int c0,
+                                                 int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+template <bool PAIR>
+__device__ __forceinline__ void tc_commit_g(uint32_t mbar) {
+  if constexpr (PAIR)
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+template <bool PAIR>
+__device__ __forceinline__ void tc_mma_g(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  if constexpr (PAIR)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc_g(uint32_t slot_saddr) {
+  if constexpr (PAIR) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_saddr),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_saddr),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_dealloc_g(uint32_t taddr) {
+  if constexpr (PAIR)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(kTmemCols) : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(kTmemCols) : "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
 // stride byte offsets (all >> 4), version 1, 128-byte swizzle (layout 2).
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -185,10 +292,10 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
   d |= (uint64_t)2 << 61;
   return d;
 }
-// Instruction descriptor, kind::f16: D fp32, A/B bf16, M=128, N=256.
-__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn_major) {
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, M = m, N = 256.
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t b_mn_major, uint32_t m) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((uint32_t)(TBN >> 3) << 17) |
-         ((uint32_t)(TBM >> 4) << 24);
+         ((m >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- scheduling
@@ -198,6 +305,10 @@ struct TileInfo {
   int g, b, m0, n0, nkb;
 };
 
+// Symmetric kinds enumerate, column block by column block, the row blocks
+// whose tile touches the upper triangle: tm <= 2 tn + 1 for 128-row tiles,
+// tm <= tn for 256-row tiles.
+template <bool PAIR>
 __device__ __forceinline__ TileInfo decode_tile(const GemmLaunch& L, int tile) {
   int g = 0;
   while (g + 1 < L.num_groups && L.g[g + 1].tile_begin <= tile) ++g;
@@ -209,20 +320,22 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmLaunch& L, int tile) {
   if (symmetric_kind(G.kind)) {
     tn = 0;
     for (;;) {
-      const int cnt = min(2 * tn + 2, G.tiles_m);
+      const int cnt = PAIR ? min(tn + 1, G.tiles_m) : min(2 * tn + 2, G.tiles_m);
       if (t < cnt) break;
       t -= cnt;
       ++tn;
     }
     tm = t;
   } else {
-    tm = t / G.tiles_n;
-    tn = t % G.tiles_n;
+    // column strips of X outermost: the concurrently running tiles share one
+    // strip of the B operand (read from HBM about once) and all of A (s x s)
+    tm = t % G.tiles_m;
+    tn = t / G.tiles_m;
   }
   TileInfo ti;
   ti.g = g;
   ti.b = b;
-  ti.m0 = tm * TBM;
+  ti.m0 = tm * Geo<PAIR>::kTileM;
   ti.n0 = tn * TBN;
   ti.nkb = (G.K + TBK - 1) / TBK;
   return ti;
@@ -231,32 +344,39 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmLaunch& L, int tile) {
 __device__ __forceinline__ float bf16_bits_to_f(uint32_t h) { return __uint_as_float(h << 16); }
 
 // ---------------------------------------------------------------- kernel
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ TcParams P) {
+  using Gm = Geo<PAIR>;
+  constexpr int S = Gm::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t sA = base;                         // STAGES x 16 KiB
-  const uint32_t sB = base + STAGES * kABytes;      // STAGES x 32 KiB
-  const uint32_t sOut = sB + STAGES * kBBytes;       // 32 KiB of output staging
-  uint8_t* ctl = smem + STAGES * kStageBytes + kOutBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);     // full[4], empty[4], tfull[2], tempty[2], drain
-  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * STAGES;
-  const uint32_t tfull0 = empty0 + 8 * STAGES, tempty0 = tfull0 + 16, drain = tempty0 + 16;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(ctl + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 132);
+  const uint32_t sA = base;                                 // S x 16 KiB
+  const uint32_t sB = base + S * Gm::kABytes;               // S x kBBytes
+  const uint32_t sOut = sB + S * Gm::kBBytes;               // 32 KiB of output staging
+  uint8_t* ctl = smem + S * Gm::kStageBytes + kOutBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);        // full[S], empty[S], tfull[2], tempty[2], drain
+  const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * S;
+  const uint32_t tfull0 = empty0 + 8 * S, tempty0 = tfull0 + 16, drain = tempty0 + 16;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(ctl + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 196);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GemmLaunch& L = P.L;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? (int)cluster_id() : (int)blockIdx.x;      // tile-processing unit
+  const int units = PAIR ? (int)cluster_count() : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 128);
+      mbar_init(tempty0 + 8 * a, (PAIR ? 2 : 1) * 4);   // one arrive per epilogue warp of each CTA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -264,20 +384,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    for (int g = 0; g < L.num_groups; ++g) {
+    for (int g = 0; g < L.num_groups; ++g)
       for (int k = 0; k < 3; ++k)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&P.maps[3 * g + k])) : "memory");
-    }
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(const_cast<uint32_t*>(tmem_slot))),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc_g<PAIR>(smem_u32(const_cast<uint32_t*>(tmem_slot)));
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();    // peer barriers initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -288,33 +402,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < L.total_tiles && ok; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(L, tile);
+      for (int tile = unit; tile < L.total_tiles && ok; tile += units) {
+        const TileInfo ti = decode_tile<PAIR>(L, tile);
         const GemmGroup& G = L.g[ti.g];
         const CUtensorMap* mA = &P.maps[3 * ti.g];
         const CUtensorMap* mB = &P.maps[3 * ti.g + 1];
         const bool upd = G.kind == GK_UPD;
+        const int arow = ti.m0 + (int)rank * 128;
+        const int bcol = ti.n0 + (int)rank * (int)Gm::kBRows;
         for (int kb = 0; kb < ti.nkb; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
-          const uint32_t fb = full0 + 8 * stage;
-          mbar_expect_tx(fb, kStageBytes);
-          tma_load_3d(sA + stage * kABytes, mA, fb, kb * TBK, ti.m0, ti.b);
-          if (upd) {
+          const uint32_t fb_local = full0 + 8 * stage;
+          if (leader) mbar_expect_tx(fb_local, Gm::kTxBytes);
+          const uint32_t fb = PAIR ? map_to_rank(fb_local, 0) : fb_local;
+          const uint32_t a_dst = sA + stage * Gm::kABytes, b_dst = sB + stage * Gm::kBBytes;
+          if constexpr (PAIR) {
+            tma_load_3d_pair(a_dst, mA, fb, kb * TBK, arow, ti.b);
+            if (upd) {
 #pragma unroll
-            for (int j = 0; j < TBN / 64; ++j)
-              tma_load_3d(sB + stage * kBBytes + j * (64 * TBK * 2), mB, fb, ti.n0 + 64 * j, kb * TBK, ti.b);
+              for (int j = 0; j < (int)Gm::kBRows / 64; ++j)
+                tma_load_3d_pair(b_dst + j * (64 * TBK * 2), mB, fb, bcol + 64 * j, kb * TBK, ti.b);
+            } else {
+              tma_load_3d_pair(b_dst, mB, fb, kb * TBK, bcol, ti.b);
+            }
           } else {
-            tma_load_3d(sB + stage * kBBytes, mB, fb, kb * TBK, ti.n0, ti.b);
+            tma_load_3d(a_dst, mA, fb, kb * TBK, arow, ti.b);
+            if (upd) {
+#pragma unroll
+              for (int j = 0; j < (int)Gm::kBRows / 64; ++j)
+                tma_load_3d(b_dst + j * (64 * TBK * 2), mB, fb, bcol + 64 * j, kb * TBK, ti.b);
+            } else {
+              tma_load_3d(b_dst, mB, fb, kb * TBK, bcol, ti.b);
+            }
           }
           ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
-        // drain: wait (bounded) for every stage's most recent load to land
-        for (uint32_t k = 0; k < STAGES && k < issued; ++k) {
+      if (!ok && leader) {
+        // drain: wait (bounded) for every stage's most recent loads (of both
+        // CTAs of a pair, which complete on this barrier) to land
+        for (uint32_t k = 0; k < (uint32_t)S && k < issued; ++k) {
           const uint32_t idx = issued - 1 - k;
-          const uint32_t st = idx % STAGES, ph = (idx / STAGES) & 1u;
+          const uint32_t st = idx % S, ph = (idx / S) & 1u;
           const long long t0 = clock64();
           while (!mbar_try_wait(full0 + 8 * st, ph) && clock64() - t0 < kWaitLimitCycles) {}
         }
@@ -322,15 +452,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, any = false;
       int it = 0;
-      for (int tile = blockIdx.x; tile < L.total_tiles && ok; tile += gridDim.x, ++it) {
-        const TileInfo ti = decode_tile(L, tile);
+      for (int tile = unit; tile < L.total_tiles && ok; tile += units, ++it) {
+        const TileInfo ti = decode_tile<PAIR>(L, tile);
         const bool upd = L.g[ti.g].kind == GK_UPD;
-        const uint32_t idesc = make_idesc(upd ? 1u : 0u);
+        const uint32_t idesc = make_idesc(upd ? 1u : 0u, (uint32_t)Gm::kTileM);
         const int acc = it & 1;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -338,24 +468,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         for (int kb = 0; kb < ti.nkb; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = sA + stage * kABytes, b0 = sB + stage * kBBytes;
+          const uint32_t a0 = sA + stage * Gm::kABytes, b0 = sB + stage * Gm::kBBytes;
 #pragma unroll
           for (int k = 0; k < TBK / 16; ++k) {
             const uint64_t ad = make_sdesc(a0 + k * 32, 16, 1024);
             const uint64_t bd = upd ? make_sdesc(b0 + k * 16 * 128, 64 * TBK * 2, 1024)
                                     : make_sdesc(b0 + k * 32, 16, 1024);
-            tc_mma(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            tc_mma_g<PAIR>(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
             any = true;
           }
-          tc_commit(empty0 + 8 * stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          tc_commit_g<PAIR>(empty0 + 8 * stage);
+          if constexpr (PAIR) tc_commit_g<PAIR>(map_to_rank(empty0 + 8 * stage, 1));
+          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(tfull0 + 8 * acc);
+        tc_commit_g<PAIR>(tfull0 + 8 * acc);
+        if constexpr (PAIR) tc_commit_g<PAIR>(map_to_rank(tfull0 + 8 * acc, 1));
         if (acc == 1) acc_phase ^= 1u;
       }
       if (!ok && any) {
-        tc_commit(drain);
+        tc_commit_g<PAIR>(drain);
         const long long t0 = clock64();
         while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles) {}
       }
@@ -369,10 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     // the diagonal is completed from its own upper triangle in shared memory.
     const int q = warp & 3;                          // TMEM lane quadrant of this warp
     const uint32_t wbuf = sOut + (uint32_t)(warp - 2) * 4u * kOutTileBytes;
+    const uint32_t tempty_leader0 = PAIR ? map_to_rank(tempty0, 0) : tempty0;
     uint32_t acc_phase = 0, par = 0;
     int it = 0;
-    for (int tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(L, tile);
+    for (int tile = unit; tile < L.total_tiles; tile += units, ++it) {
+      const TileInfo ti = decode_tile<PAIR>(L, tile);
       const GemmGroup& G = L.g[ti.g];
       const int acc = it & 1;
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
@@ -383,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         for (int p = 0; p < G.pa; ++p) alpha *= r;
         for (int p = 0; p < G.pb; ++p) beta *= r;
       }
-      const int r0 = ti.m0 + q * 32;                 // first row of this warp's strip
+      const int r0 = ti.m0 + (int)rank * 128 + q * 32;   // first row of this warp's strip
       const int row = r0 + lane;
       const bool sym = symmetric_kind(G.kind);
       const CUtensorMap* mC = &P.maps[3 * ti.g + 2];
@@ -456,8 +589,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         }
         par ^= 1u;
       }
+      // this warp's TMEM reads of the accumulator are complete: release it
       tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+        else mbar_arrive(tempty0 + 8 * acc);
+      }
       if (acc == 1) acc_phase ^= 1u;
     }
     if (lane == 0) bulk_wait_all();
@@ -466,10 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // the leader's MMAs write the peer's TMEM: free it only after both are done
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
-                 : "memory");
+    tmem_dealloc_g<PAIR>(tmem_base);
   }
 }
 
@@ -502,6 +640,50 @@ bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uin
   return r == CUDA_SUCCESS;
 }
 
+// Per-device launch facts for one kernel variant: the shared-memory opt-in
+// and the number of CTA pairs that can be resident at once.
+struct DeviceFacts {
+  cudaError_t err = cudaSuccess;
+  int units = 0;
+};
+
+template <bool PAIR>
+DeviceFacts device_facts(int num_sms) {
+  static std::mutex mu;
+  static std::map<int, DeviceFacts> cache;
+  int dev = 0;
+  DeviceFacts f;
+  if ((f.err = cudaGetDevice(&dev)) != cudaSuccess) return f;
+  std::lock_guard<std::mutex> g(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  f.err = cudaFuncSetAttribute(k_gemm_tc<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)Geo<PAIR>::kSmemBytes);
+  if (f.err == cudaSuccess) {
+    if constexpr (PAIR) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = Geo<PAIR>::kSmemBytes;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      f.err = cudaOccupancyMaxActiveClusters(&clusters, k_gemm_tc<PAIR>, &cfg);
+      f.units = clusters;
+    } else {
+      f.units = num_sms;
+    }
+  }
+  if (f.err == cudaSuccess && f.units <= 0) f.err = cudaErrorInvalidConfiguration;
+  cache[dev] = f;
+  return f;
+}
+
 }  // namespace
 
 cudaError_t read_and_clear_device_status(unsigned int* out) {
@@ -513,26 +695,28 @@ cudaError_t read_and_clear_device_status(unsigned int* out) {
   return e;
 }
 
-int tc_tile_count(int kind, int M, int N, int* tiles_m, int* tiles_n) {
-  const int tm = (M + TBM - 1) / TBM, tn = (N + TBN - 1) / TBN;
+int tc_tile_count(int kind, int M, int N, bool pair, int* tiles_m, int* tiles_n) {
+  const int tile_m = pair ? 256 : 128;
+  const int tm = (M + tile_m - 1) / tile_m, tn = (N + TBN - 1) / TBN;
   *tiles_m = tm;
   *tiles_n = tn;
   if (kind == GK_UPD) return tm * tn;
   int c = 0;
-  for (int j = 0; j < tn; ++j) c += std::min(2 * j + 2, tm);
+  for (int j = 0; j < tn; ++j) c += std::min(pair ? j + 1 : 2 * j + 2, tm);
   return c;
 }
 
-bool tc_encode_maps(const GemmLaunch& L, void* maps_out) {
+bool tc_encode_maps(const GemmLaunch& L, bool pair, void* maps_out) {
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_out);
+  const uint32_t brows = pair ? 128 : 256;
   for (int g = 0; g < L.num_groups; ++g) {
     const GemmGroup& G = L.g[g];
-    if (!encode_3d(&maps[3 * g], G.A, G.K, G.M, G.count, G.lda, G.sa, TBK, TBM)) return false;
+    if (!encode_3d(&maps[3 * g], G.A, G.K, G.M, G.count, G.lda, G.sa, TBK, 128)) return false;
     bool ok;
     if (G.kind == GK_UPD)
       ok = encode_3d(&maps[3 * g + 1], G.B, G.N, G.K, G.count, G.ldb, G.sb, 64, TBK);
     else
-      ok = encode_3d(&maps[3 * g + 1], G.B, G.K, G.N, G.count, G.ldb, G.sb, TBK, TBN);
+      ok = encode_3d(&maps[3 * g + 1], G.B, G.K, G.N, G.count, G.ldb, G.sb, TBK, brows);
     if (!ok) return false;
     if (!encode_3d(&maps[3 * g + 2], G.C, G.N, G.M, G.count, G.ldc, G.sc, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return false;
@@ -540,21 +724,38 @@ bool tc_encode_maps(const GemmLaunch& L, void* maps_out) {
   return true;
 }
 
-cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, cudaStream_t st) {
+cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, bool pair, cudaStream_t st) {
   if (L.total_tiles == 0) return cudaSuccess;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
   TcParams* P = new TcParams;
   std::memcpy(P->maps, maps, sizeof(CUtensorMap) * 3 * L.num_groups);
   P->L = L;
-  const int grid = std::min(num_sms, L.total_tiles);
-  k_gemm_tc<<<grid, kThreads, kSmemBytes, st>>>(*P);
+  cudaError_t e;
+  if (pair) {
+    const DeviceFacts f = device_facts<true>(num_sms);
+    if (f.err != cudaSuccess) { delete P; return f.err; }
+    const int clusters = std::min(f.units, L.total_tiles);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Geo<true>::kSmemBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_gemm_tc<true>, *P);
+  } else {
+    const DeviceFacts f = device_facts<false>(num_sms);
+    if (f.err != cudaSuccess) { delete P; return f.err; }
+    const int grid = std::min(f.units, L.total_tiles);
+    k_gemm_tc<false><<<grid, kThreads, Geo<false>::kSmemBytes, st>>>(*P);
+    e = cudaGetLastError();
+  }
   delete P;
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace am

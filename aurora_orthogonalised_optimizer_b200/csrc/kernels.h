@@ -47,10 +47,10 @@ cudaError_t launch_gemm_simt(const GemmLaunch& L, cudaStream_t st);
 
 // tcgen05 grouped GEMM (bf16 operands, fp32 accumulation in TMEM, TMA loads).
 // `maps` holds three CUtensorMap (128 B each) per group: operand A, operand B, output C.
-struct TcLaunch;
-cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, cudaStream_t st);
-bool tc_encode_maps(const GemmLaunch& L, void* maps_out);  // host: builds the tensor maps
-int tc_tile_count(int kind, int M, int N, int* tiles_m, int* tiles_n);
+// `pair` selects the SM-pair variant (clusters of two CTAs, 256 x 256 tiles).
+cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, bool pair, cudaStream_t st);
+bool tc_encode_maps(const GemmLaunch& L, bool pair, void* maps_out);  // host: builds the tensor maps
+int tc_tile_count(int kind, int M, int N, bool pair, int* tiles_m, int* tiles_n);
 cudaError_t read_and_clear_device_status(unsigned int* out);  // current device
 
 // ---------------------------------------------------------------- element-wise
