@@ -289,6 +289,7 @@ k_matvec(const MatTable t, int dir) {
     const int64_t i = (int64_t)b * 8 + w;
     if (i < d.s) {
       float acc = 0.f;
+#pragma unroll 4
       for (int64_t j = 8 * lane; j < d.l; j += 256) {
         float x[8], v[8];
         ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);

@@ -1,0 +1,76 @@
+"""Full-size parity of the 3.8B matrix set (168 matrices, 2.82 G parameters)
+in the launch configuration the bench times: one muon_step call over every
+matrix, tensor-core Newton-Schulz.
+
+* Sampled outputs: the k and v matrices (1024 x 3072) of the first and the
+  last layer are recomputed by the float64 oracle; update V within 3e-2
+  relative Frobenius error, momentum within 1e-6.
+* Properties that hold for every matrix at any size, checked on all 168:
+  - first step from zero momentum: m = (1 - mu) g up to fp32 rounding;
+  - the parameter add: W_new = W - lr V up to the bf16 rounding of W_new
+    and the fp32 rounding of the product and the difference;
+  - the update is finite and (Aurora stack) ||V||_F / ||W||_F >= TARGET_UW.
+"""
+import numpy as np
+import pytest
+
+import oracle.muon_oracle as O
+import workloads as WL
+from tests.helpers import f64, rel_fro
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+from aurora_orthogonalised_optimizer_b200 import _abi as A  # noqa: E402
+
+
+def _run(wl, sample):
+    W, G = WL.generate_torch(wl, None, 0, threads=16)
+    cfg = A.Config.from_step_config(wl.cfg, gemm_mode=A.MUON_GEMM_BF16, param_dtype=A.MUON_BF16,
+                                    grad_dtype=A.MUON_BF16)
+    p = [w.cuda() for w in W]
+    g = [x.cuda() for x in G]
+    m = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    v = [torch.empty(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    w_before = [t.clone() for t in p]
+    ws = A.make_workspace(cfg, wl.shapes)
+    A.muon_step(cfg, p, g, m, v, ws)
+    torch.cuda.synchronize()
+    assert A.last_device_status() == A.MUON_OK
+    del ws
+    mu, lr = wl.cfg.mu, wl.cfg.lr
+    for k in range(wl.n):
+        gk = g[k].float()
+        assert torch.isfinite(v[k]).all()
+        em = ((m[k] - (1.0 - mu) * gk).norm() / ((1.0 - mu) * gk).norm()).item()
+        assert em <= 1e-6, ("momentum", k, em)
+        w0 = w_before[k].double()
+        step = lr * v[k].double()
+        want = w0 - step
+        # bf16 rounding of W_new plus the fp32 rounding of lr * V and of the subtraction
+        half_ulp = torch.ldexp(torch.ones_like(want), torch.frexp(want.abs().clamp_min(1e-30))[1] - 9)
+        bound = 1.01 * half_ulp + 2.0 ** -23 * (step.abs() + want.abs())
+        err = (p[k].double() - want).abs()
+        assert bool((err <= bound).all()), ("param add", k, (err / bound).max().item())
+        if wl.cfg.target_uw > 0:
+            assert (v[k].norm() / w0.norm()).item() >= wl.cfg.target_uw * (1 - 1e-5)
+    # sampled matrices against the oracle
+    for k in sample:
+        Wn, Gn, Mn = WL.generate(wl, [k])
+        _, m_or, V_or = O.step(WL.to_f64(Wn[0], WL.BF16), WL.to_f64(Gn[0], WL.BF16), Mn[0].astype(np.float64),
+                               wl.cfg, WL.BF16)
+        ev = rel_fro(f64(v[k]), V_or)
+        assert ev <= 3e-2, ("V", k, wl.shapes[k], ev)
+        assert rel_fro(f64(m[k]), m_or) <= 1e-6
+
+
+def test_llama_3p8b_aurora_stack_full_size():
+    wl = WL.llama_3p8b_aurora()
+    # k, v of layer 0 and of layer 27 (1024 x 3072, the Aurora wide path)
+    _run(wl, [1, 2, 6 * 27 + 1, 6 * 27 + 2])
+
+
+def test_llama_3p8b_plain_muon_full_size():
+    wl = WL.llama_3p8b_plain()
+    _run(wl, [1, 6 * 27 + 2])
