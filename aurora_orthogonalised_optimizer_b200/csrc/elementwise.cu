@@ -45,72 +45,76 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
   __shared__ float tile[kTile][kTile + 1];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
-  const int b = blockIdx.x - t.blk_prefix[mi];
-  const int64_t tiles_c = (d.n + kTile - 1) / kTile;
-  const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
-  const bool vec = (d.n & 7) == 0;
-  const bool xvec = (d.ldl & 7) == 0;
-  const int64_t j = c0 + 8 * cg;
-  const bool in0 = r0 + rg < d.m && j < d.n, in1 = r0 + rg + 32 < d.m && j < d.n;
-  const int64_t ro0 = (r0 + rg) * d.n, ro1 = (r0 + rg + 32) * d.n;
-  float g0[8], g1[8], m0[8], m1[8], w0[8], w1[8];
+  const int nt = (int)(((d.m + kTile - 1) / kTile) * ((d.n + kTile - 1) / kTile));
+  const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int b = b0; b < b0 + kEwTilesPerCta && b < nt; ++b) {
+    if (b != b0) __syncthreads();   // shared tile reused by the next tile
+    const int64_t tiles_c = (d.n + kTile - 1) / kTile;
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+    const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+    const bool vec = (d.n & 7) == 0;
+    const bool xvec = (d.ldl & 7) == 0;
+    const int64_t j = c0 + 8 * cg;
+    const bool in0 = r0 + rg < d.m && j < d.n, in1 = r0 + rg + 32 < d.m && j < d.n;
+    const int64_t ro0 = (r0 + rg) * d.n, ro1 = (r0 + rg + 32) * d.n;
+    float g0[8], g1[8], m0[8], m1[8], w0[8], w1[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) g0[e] = g1[e] = m0[e] = m1[e] = w0[e] = w1[e] = 0.f;
-  if (in0) ld8r(d.G, ro0, j, d.n, vec, t.grad_dtype, g0);
-  if (in1) ld8r(d.G, ro1, j, d.n, vec, t.grad_dtype, g1);
-  if (mode == 0) {
-    if (in0) ld8r(d.M, ro0, j, d.n, vec, kF32, m0);
-    if (in1) ld8r(d.M, ro1, j, d.n, vec, kF32, m1);
-    if (want_w2) {
-      if (in0) ld8r(d.W, ro0, j, d.n, vec, t.param_dtype, w0);
-      if (in1) ld8r(d.W, ro1, j, d.n, vec, t.param_dtype, w1);
-    }
-  }
-  float su2 = 0.f, sw2 = 0.f;
-  float u0[8], u1[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < 8; ++e) g0[e] = g1[e] = m0[e] = m1[e] = w0[e] = w1[e] = 0.f;
+    if (in0) ld8r(d.G, ro0, j, d.n, vec, t.grad_dtype, g0);
+    if (in1) ld8r(d.G, ro1, j, d.n, vec, t.grad_dtype, g1);
     if (mode == 0) {
-      m0[e] = m0[e] + (1.f - mu) * (g0[e] - m0[e]);
-      m1[e] = m1[e] + (1.f - mu) * (g1[e] - m1[e]);
-      u0[e] = nesterov ? g0[e] + mu * (m0[e] - g0[e]) : m0[e];
-      u1[e] = nesterov ? g1[e] + mu * (m1[e] - g1[e]) : m1[e];
-    } else {
-      u0[e] = g0[e];
-      u1[e] = g1[e];
-    }
-    su2 += u0[e] * u0[e] + u1[e] * u1[e];
-    sw2 += w0[e] * w0[e] + w1[e] * w1[e];
-  }
-  if (mode == 0) {
-    if (in0) st8r(d.M, ro0, j, d.n, vec, kF32, m0);
-    if (in1) st8r(d.M, ro1, j, d.n, vec, kF32, m1);
-  }
-  if (!d.tall) {
-    if (in0) st8r(d.uX, (r0 + rg) * d.ldl, j, d.n, xvec, t.ns_dtype, u0);
-    if (in1) st8r(d.uX, (r0 + rg + 32) * d.ldl, j, d.n, xvec, t.ns_dtype, u1);
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      tile[rg][8 * cg + e] = u0[e];
-      tile[rg + 32][8 * cg + e] = u1[e];
-    }
-    __syncthreads();
-    // X row = original column c0 + xr; X columns = original rows r0 + 8 cg ..
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int xr = rg + 32 * k;
-      const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
-      if (xi < d.n && xj < d.m) {
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = tile[8 * cg + e][xr];
-        st8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, v);
+      if (in0) ld8r(d.M, ro0, j, d.n, vec, kF32, m0);
+      if (in1) ld8r(d.M, ro1, j, d.n, vec, kF32, m1);
+      if (want_w2) {
+        if (in0) ld8r(d.W, ro0, j, d.n, vec, t.param_dtype, w0);
+        if (in1) ld8r(d.W, ro1, j, d.n, vec, t.param_dtype, w1);
       }
     }
+    float su2 = 0.f, sw2 = 0.f;
+    float u0[8], u1[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (mode == 0) {
+        m0[e] = m0[e] + (1.f - mu) * (g0[e] - m0[e]);
+        m1[e] = m1[e] + (1.f - mu) * (g1[e] - m1[e]);
+        u0[e] = nesterov ? g0[e] + mu * (m0[e] - g0[e]) : m0[e];
+        u1[e] = nesterov ? g1[e] + mu * (m1[e] - g1[e]) : m1[e];
+      } else {
+        u0[e] = g0[e];
+        u1[e] = g1[e];
+      }
+      su2 += u0[e] * u0[e] + u1[e] * u1[e];
+      sw2 += w0[e] * w0[e] + w1[e] * w1[e];
+    }
+    if (mode == 0) {
+      if (in0) st8r(d.M, ro0, j, d.n, vec, kF32, m0);
+      if (in1) st8r(d.M, ro1, j, d.n, vec, kF32, m1);
+    }
+    if (!d.tall) {
+      if (in0) st8r(d.uX, (r0 + rg) * d.ldl, j, d.n, xvec, t.ns_dtype, u0);
+      if (in1) st8r(d.uX, (r0 + rg + 32) * d.ldl, j, d.n, xvec, t.ns_dtype, u1);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        tile[rg][8 * cg + e] = u0[e];
+        tile[rg + 32][8 * cg + e] = u1[e];
+      }
+      __syncthreads();
+      // X row = original column c0 + xr; X columns = original rows r0 + 8 cg ..
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int xr = rg + 32 * k;
+        const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
+        if (xi < d.n && xj < d.m) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = tile[8 * cg + e][xr];
+          st8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, v);
+        }
+      }
+    }
+    warp_partials(partials, d.part + b, 2, su2, sw2);
   }
-  warp_partials(partials, d.part + b, 2, su2, sw2);
 }
 
 // Sum the per-warp partials of each matrix into its scalar block.  Layout:
@@ -182,30 +186,33 @@ __global__ void __launch_bounds__(kEwThreads)
 k_scale_cols(const MatTable t, double* partials) {
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
-  const int b = blockIdx.x - t.blk_prefix[mi];
-  const int64_t tiles_c = (d.l + kTile - 1) / kTile;
-  const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
-  const int64_t j = c0 + 8 * cg;
-  const bool vec = (d.ldl & 7) == 0;
-  float s2 = 0.f;
-  if (j < d.l) {
-    const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
-    const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
-    float dj[8], x0[8], x1[8];
-    ld8r(d.D, 0, j, d.l, true, kF32, dj);
-    if (in0) ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, x0);
-    if (in1) ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, x1);
+  const int nt = (int)(((d.s + kTile - 1) / kTile) * ((d.l + kTile - 1) / kTile));
+  const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int b = b0; b < b0 + kEwTilesPerCta && b < nt; ++b) {
+    const int64_t tiles_c = (d.l + kTile - 1) / kTile;
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+    const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+    const int64_t j = c0 + 8 * cg;
+    const bool vec = (d.ldl & 7) == 0;
+    float s2 = 0.f;
+    if (j < d.l) {
+      const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
+      const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
+      float dj[8], x0[8], x1[8];
+      ld8r(d.D, 0, j, d.l, true, kF32, dj);
+      if (in0) ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, x0);
+      if (in1) ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, x1);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      x0[e] = in0 ? x0[e] * dj[e] : 0.f;
-      x1[e] = in1 ? x1[e] * dj[e] : 0.f;
-      s2 += x0[e] * x0[e] + x1[e] * x1[e];
+      for (int e = 0; e < 8; ++e) {
+        x0[e] = in0 ? x0[e] * dj[e] : 0.f;
+        x1[e] = in1 ? x1[e] * dj[e] : 0.f;
+        s2 += x0[e] * x0[e] + x1[e] * x1[e];
+      }
+      if (in0) st8r(d.X0, ro0, j, d.l, vec, t.ns_dtype, x0);
+      if (in1) st8r(d.X0, ro1, j, d.l, vec, t.ns_dtype, x1);
     }
-    if (in0) st8r(d.X0, ro0, j, d.l, vec, t.ns_dtype, x0);
-    if (in1) st8r(d.X0, ro1, j, d.l, vec, t.ns_dtype, x1);
+    warp_partials(partials, d.part + b, 1, s2, 0.f);
   }
-  warp_partials(partials, d.part + b, 1, s2, 0.f);
 }
 
 // Per-matrix scalar algebra (one thread per matrix).
@@ -269,7 +276,7 @@ __global__ void k_scalars(const MatTable t, int op, int src_slot, float ns_eps, 
 // Power iteration ("组合优化栈": scale_to_unit_operator_norm, 5 iterations).
 // On the X orientation Q (s x l):
 //   flag 0 (row dot):  out_i = sum_j Q_ij x_j   (x length l, out length s)
-//                      one warp per row, 8-element groups per lane
+//                      one warp per kMatvecRowsPerWarp rows, 8-element groups per lane
 //   flag 1 (col dot):  out_j = sum_i Q_ij y_i   (y length s, out length l)
 //                      64 columns per block, 8 groups x 32 row lanes
 // `dir` selects vec0 -> vec1 (0) or vec1 -> vec0 (1).  The vectors are
@@ -285,20 +292,31 @@ k_matvec(const MatTable t, int dir) {
   float* out = dir == 0 ? d.vec1 : d.vec0;
   const bool vec = (d.ldl & 7) == 0;
   if (d.flag == 0) {
+    // each warp reduces kMatvecRowsPerWarp rows, loading the vector chunk once
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int64_t i = (int64_t)b * 8 + w;
-    if (i < d.s) {
-      float acc = 0.f;
-#pragma unroll 4
+    const int64_t i0 = (int64_t)b * kMatvecRowsPerCta + w * kMatvecRowsPerWarp;
+    float acc[kMatvecRowsPerWarp];
+#pragma unroll
+    for (int r = 0; r < kMatvecRowsPerWarp; ++r) acc[r] = 0.f;
+    if (i0 < d.s) {
       for (int64_t j = 8 * lane; j < d.l; j += 256) {
-        float x[8], v[8];
-        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+        float v[8];
         ld8r(in, 0, j, d.l, true, kF32, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc += x[e] * v[e];
+        for (int r = 0; r < kMatvecRowsPerWarp; ++r) {
+          if (i0 + r < d.s) {
+            float x[8];
+            ld8r(d.uX, (i0 + r) * d.ldl, j, d.l, vec, t.ns_dtype, x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[r] += x[e] * v[e];
+          }
+        }
       }
-      acc = warp_sum(acc);
-      if (lane == 0) out[i] = acc;
+#pragma unroll
+      for (int r = 0; r < kMatvecRowsPerWarp; ++r) {
+        const float a = warp_sum(acc[r]);
+        if (lane == 0 && i0 + r < d.s) out[i0 + r] = a;
+      }
     }
   } else {
     const int cg = threadIdx.x & 7, rl = threadIdx.x >> 3;
@@ -362,28 +380,31 @@ __global__ void __launch_bounds__(kEwThreads)
 k_dots(const MatTable t, double* partials) {
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
-  const int b = blockIdx.x - t.blk_prefix[mi];
-  const int64_t tiles_c = (d.l + kTile - 1) / kTile;
-  const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
-  const int64_t j = c0 + 8 * cg;
-  const bool vec = (d.ldl & 7) == 0;
-  float a = 0.f, c = 0.f;
-  if (j < d.l) {
-    const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
-    const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
-    float U0[8], u0[8], U1[8], u1[8];
+  const int nt = (int)(((d.s + kTile - 1) / kTile) * ((d.l + kTile - 1) / kTile));
+  const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int b = b0; b < b0 + kEwTilesPerCta && b < nt; ++b) {
+    const int64_t tiles_c = (d.l + kTile - 1) / kTile;
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+    const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+    const int64_t j = c0 + 8 * cg;
+    const bool vec = (d.ldl & 7) == 0;
+    float a = 0.f, c = 0.f;
+    if (j < d.l) {
+      const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
+      const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
+      float U0[8], u0[8], U1[8], u1[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) U0[e] = u0[e] = U1[e] = u1[e] = 0.f;
-    if (in0) { ld8r(d.UX, ro0, j, d.l, vec, t.ns_dtype, U0); ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, u0); }
-    if (in1) { ld8r(d.UX, ro1, j, d.l, vec, t.ns_dtype, U1); ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, u1); }
+      for (int e = 0; e < 8; ++e) U0[e] = u0[e] = U1[e] = u1[e] = 0.f;
+      if (in0) { ld8r(d.UX, ro0, j, d.l, vec, t.ns_dtype, U0); ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, u0); }
+      if (in1) { ld8r(d.UX, ro1, j, d.l, vec, t.ns_dtype, U1); ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, u1); }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      a += U0[e] * U0[e] + U1[e] * U1[e];
-      c += U0[e] * u0[e] + U1[e] * u1[e];
+      for (int e = 0; e < 8; ++e) {
+        a += U0[e] * U0[e] + U1[e] * U1[e];
+        c += U0[e] * u0[e] + U1[e] * u1[e];
+      }
     }
+    warp_partials(partials, d.part + b, 2, a, c);
   }
-  warp_partials(partials, d.part + b, 2, a, c);
 }
 
 // ============================================================================
@@ -398,69 +419,73 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
   __shared__ float tu[kTile][kTile + 1];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
-  const int b = blockIdx.x - t.blk_prefix[mi];
-  const int64_t tiles_c = (d.n + kTile - 1) / kTile;
-  const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
-  const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
-  const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
-  const bool need_U = cU != 0.f, need_u = cu != 0.f;
-  const bool vec = (d.n & 7) == 0;
-  const bool xvec = (d.ldl & 7) == 0;
-  if (d.tall) {
-    // X tile rows = original columns c0 + xr, X tile columns = original rows r0 + 8 cg ..
+  const int nt = (int)(((d.m + kTile - 1) / kTile) * ((d.n + kTile - 1) / kTile));
+  const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int b = b0; b < b0 + kEwTilesPerCta && b < nt; ++b) {
+    if (b != b0) __syncthreads();   // shared tile reused by the next tile
+    const int64_t tiles_c = (d.n + kTile - 1) / kTile;
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+    const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+    const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
+    const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
+    const bool need_U = cU != 0.f, need_u = cu != 0.f;
+    const bool vec = (d.n & 7) == 0;
+    const bool xvec = (d.ldl & 7) == 0;
+    if (d.tall) {
+      // X tile rows = original columns c0 + xr, X tile columns = original rows r0 + 8 cg ..
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int xr = rg + 32 * k;
+        const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
+        float U[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (xi < d.n && xj < d.m) {
+          if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, U);
+          if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, u);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          tU[xr][8 * cg + e] = U[e];
+          tu[xr][8 * cg + e] = u[e];
+        }
+      }
+      __syncthreads();
+    }
+    const int64_t j = c0 + 8 * cg;
+    float U[2][8], u[2][8], w[2][8];
+    bool in[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int xr = rg + 32 * k;
-      const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
-      float U[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (xi < d.n && xj < d.m) {
-        if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, U);
-        if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, u);
+      const int rr = rg + 32 * k;
+      const int64_t i = r0 + rr;
+      in[k] = i < d.m && j < d.n;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) U[k][e] = u[k][e] = w[k][e] = 0.f;
+      if (!in[k]) continue;
+      if (d.tall) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          U[k][e] = tU[8 * cg + e][rr];
+          u[k][e] = tu[8 * cg + e][rr];
+        }
+      } else {
+        if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U[k]);
+        if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u[k]);
       }
+      if (update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!in[k]) continue;
+      const int64_t ro = (r0 + rg + 32 * k) * d.n;
+      float v[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        tU[xr][8 * cg + e] = U[e];
-        tu[xr][8 * cg + e] = u[e];
+        v[e] = cU * U[k][e] + cu * u[k][e];
+        w[k][e] -= lr * v[e];
       }
+      if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v);
+      if (update_w) st8r(d.W, ro, j, d.n, vec, t.param_dtype, w[k]);
     }
-    __syncthreads();
-  }
-  const int64_t j = c0 + 8 * cg;
-  float U[2][8], u[2][8], w[2][8];
-  bool in[2];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int rr = rg + 32 * k;
-    const int64_t i = r0 + rr;
-    in[k] = i < d.m && j < d.n;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) U[k][e] = u[k][e] = w[k][e] = 0.f;
-    if (!in[k]) continue;
-    if (d.tall) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        U[k][e] = tU[8 * cg + e][rr];
-        u[k][e] = tu[8 * cg + e][rr];
-      }
-    } else {
-      if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U[k]);
-      if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u[k]);
-    }
-    if (update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    if (!in[k]) continue;
-    const int64_t ro = (r0 + rg + 32 * k) * d.n;
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      v[e] = cU * U[k][e] + cu * u[k][e];
-      w[k][e] -= lr * v[e];
-    }
-    if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v);
-    if (update_w) st8r(d.W, ro, j, d.n, vec, t.param_dtype, w[k]);
   }
 }
 

@@ -301,6 +301,9 @@ double table_elems(const MatTable& t) {
 
 int64_t tiles_orig(const MatDesc& d) { return cdiv(d.m, 64) * cdiv(d.n, 64); }
 int64_t tiles_x(const MatDesc& d) { return cdiv(d.s, 64) * cdiv(d.l, 64); }
+// blocks of a streaming launch (kEwTilesPerCta tiles each)
+int64_t blocks_orig(const MatDesc& d) { return cdiv(tiles_orig(d), kEwTilesPerCta); }
+int64_t blocks_x(const MatDesc& d) { return cdiv(tiles_x(d), kEwTilesPerCta); }
 
 #define CK(expr)                                   \
   do {                                             \
@@ -312,7 +315,7 @@ int64_t tiles_x(const MatDesc& d) { return cdiv(d.s, 64) * cdiv(d.l, 64); }
 muon_status stage_prologue(const Ctx& c, const std::vector<int>& ids, int mode, bool want_w2) {
   const double per_elem = dt_bytes(c.grad_dtype) + c.plan->nsb + (mode == 0 ? 8.0 : 0.0) +
                           (want_w2 ? dt_bytes(c.param_dtype) : 0.0);
-  CK(for_chunks(c, ids, tiles_orig, [&](const MatTable& t, int nb) {
+  CK(for_chunks(c, ids, blocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_prologue(t, nb, mode, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
   }));
@@ -340,7 +343,7 @@ muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int
     return for_chunks(c, ids, [first](MatDesc& d) -> int64_t {
       const bool rowdot = first ? !d.tall : (bool)d.tall;
       d.flag = rowdot ? 0 : 1;
-      return rowdot ? cdiv(d.s, 8) : cdiv(d.l, 64);
+      return rowdot ? cdiv(d.s, kMatvecRowsPerCta) : cdiv(d.l, 64);
     }, [&](const MatTable& t, int nb) {
       ProfScope ps(PC_POWER, 2.0 * table_elems(t), c.plan->nsb * table_elems(t), c.st);
       return launch_matvec(t, nb, dir, c.st);
@@ -506,7 +509,7 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
   const int rounds = eq_b.empty() ? 1 : c.cfg->pp_iterations;
   for (int k = 0; k < rounds; ++k) {
     if (!eq_ids.empty()) {
-      CK(for_chunks(c, eq_ids, tiles_x, [&](const MatTable& t, int nb) {
+      CK(for_chunks(c, eq_ids, blocks_x, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
         return launch_scale_cols(t, nb, c.partials, c.st);
       }));
@@ -545,7 +548,7 @@ muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool updat
   const bool need_u = c.cfg->contra != 0.f || !update_w;
   const double per_elem = c.plan->nsb * (need_u ? 2.0 : 1.0) + (update_w ? 2.0 * dt_bytes(c.param_dtype) : 0.0) +
                           (c.V ? 4.0 : 0.0);
-  CK(for_chunks(c, ids, tiles_orig, [&](const MatTable& t, int nb) {
+  CK(for_chunks(c, ids, blocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_epilogue(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
   }));
@@ -553,7 +556,7 @@ muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool updat
 }
 
 muon_status stage_dots(const Ctx& c, const std::vector<int>& ids) {
-  CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int nb) {
+  CK(for_chunks(c, ids, blocks_x, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_REDUCE, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
     return launch_dots(t, nb, c.partials, c.st);
   }));

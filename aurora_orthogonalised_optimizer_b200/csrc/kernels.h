@@ -54,6 +54,13 @@ int tc_tile_count(int kind, int M, int N, bool pair, int* tiles_m, int* tiles_n)
 cudaError_t read_and_clear_device_status(unsigned int* out);  // current device
 
 // ---------------------------------------------------------------- element-wise
+// Streaming kernels work on 64 x 64 tiles; a block walks kEwTilesPerCta
+// consecutive tiles of one matrix (launch ceil(tiles / kEwTilesPerCta)
+// blocks per matrix); reductions still leave one set of partials per tile.
+constexpr int kEwTilesPerCta = 4;
+// Row-dot pass of the power iteration: 8 warps x kMatvecRowsPerWarp rows.
+constexpr int kMatvecRowsPerWarp = 4;
+constexpr int kMatvecRowsPerCta = 8 * kMatvecRowsPerWarp;
 cudaError_t launch_prologue(const MatTable& t, int nblk, int mode, float mu, int nesterov,
                             int want_w2, double* partials, cudaStream_t st);
 cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int nq, int slot0,

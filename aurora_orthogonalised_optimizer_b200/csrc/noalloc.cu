@@ -115,7 +115,8 @@ extern "C" muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, c
       for (int k = 0; k < cnt; ++k) {
         MatDesc& d = t.mats[k];
         d.flag = pass == 2 ? 1 : 0;
-        d.nblk = pass == 1 ? (int)((d.s + 7) / 8) : pass == 2 ? (int)((d.l + 63) / 64) : 0;
+        d.nblk = pass == 1 ? (int)((d.s + kMatvecRowsPerCta - 1) / kMatvecRowsPerCta)
+                 : pass == 2 ? (int)((d.l + 63) / 64) : 0;
         t.blk_prefix[k] = tot;
         tot += d.nblk;
       }
@@ -143,7 +144,7 @@ extern "C" muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, c
       int tiles = 0;
       for (int k = 0; k < cnt; ++k) {
         MatDesc& d = t.mats[k];
-        d.nblk = (int)(((d.m + 63) / 64) * ((d.n + 63) / 64));
+        d.nblk = (int)((((d.m + 63) / 64) * ((d.n + 63) / 64) + kEwTilesPerCta - 1) / kEwTilesPerCta);
         t.blk_prefix[k] = tiles;
         tiles += d.nblk;
       }
