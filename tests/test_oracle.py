@@ -324,3 +324,33 @@ def test_workload_constants_match_pages():
     assert c.lr == g["lr_aurora"]["value"]
     assert sum(m * n for m, n in WL.llama_3p8b_shapes()) == 2_818_572_288
     assert len(WL.gpt2_124m_shapes()) == 72
+
+
+# --------------------------------------------------------------- auxiliary AdamW
+def test_adamw_constant_gradient_closed_form():
+    """Constant g from zero state: m_hat = g, v_hat = g^2, so each step moves lr g/(|g| + eps)."""
+    rng = np.random.default_rng(30)
+    g = rng.standard_normal(50) + 0.5
+    p0 = rng.standard_normal(50)
+    p, m, v = p0.copy(), np.zeros(50), np.zeros(50)
+    lr, eps = 0.01, 1e-10
+    for t in range(1, 8):
+        p, m, v = O.adamw_step(p, g, m, v, lr, 0.8, 0.95, eps, 0.0, t)
+        assert np.allclose(m, (1 - 0.8 ** t) * g, rtol=1e-13)
+        assert np.allclose(v, (1 - 0.95 ** t) * g * g, rtol=1e-13)
+        assert np.allclose(p, p0 - t * lr * g / (np.abs(g) + eps), rtol=1e-12, atol=1e-14)
+
+
+def test_adamw_matches_torch_adamw_float64():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(31)
+    p0 = rng.standard_normal((7, 5))
+    grads = [rng.standard_normal((7, 5)) for _ in range(4)]
+    tp = torch.tensor(p0, dtype=torch.float64, requires_grad=True)
+    opt = torch.optim.AdamW([tp], lr=0.3, betas=(0.8, 0.95), eps=1e-10, weight_decay=0.05)
+    p, m, v = p0.copy(), np.zeros_like(p0), np.zeros_like(p0)
+    for t, g in enumerate(grads, start=1):
+        tp.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        p, m, v = O.adamw_step(p, g, m, v, 0.3, 0.8, 0.95, 1e-10, 0.05, t)
+        assert np.allclose(p, tp.detach().numpy(), rtol=1e-12, atol=1e-14)
