@@ -23,7 +23,8 @@ MUON_GEMM_BF16, MUON_GEMM_FP32, MUON_GEMM_BF16_SIMT = 0, 1, 2
 
 EXPORTS = ["muon_config_default", "muon_workspace_size", "muon_step", "ns_polar", "aurora_polar",
            "opnorm_normalize", "uw_floor_apply", "muon_last_device_status", "muon_status_string",
-           "muon_profile_enable", "muon_profile_read", "opnorm_normalize_noalloc"]
+           "muon_profile_enable", "muon_profile_read", "opnorm_normalize_noalloc",
+           "adamw_config_default", "adamw_step"]
 
 
 class MuonShape(C.Structure):
@@ -40,6 +41,12 @@ class MuonConfig(C.Structure):
         ("target_uw", C.c_float), ("weight_decay", C.c_float),
         ("gemm_mode", C.c_int), ("param_dtype", C.c_int), ("grad_dtype", C.c_int),
     ]
+
+
+class AdamWConfig(C.Structure):
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
+                ("weight_decay", C.c_float), ("step", C.c_int), ("param_dtype", C.c_int),
+                ("grad_dtype", C.c_int)]
 
 
 class MuonProfileEntry(C.Structure):
@@ -91,6 +98,11 @@ def load():
     lib.muon_last_device_status.restype = C.c_int
     lib.muon_status_string.argtypes = [C.c_int]
     lib.muon_status_string.restype = C.c_char_p
+    lib.adamw_config_default.argtypes = [C.POINTER(AdamWConfig)]
+    lib.adamw_config_default.restype = None
+    lib.adamw_step.argtypes = [C.POINTER(AdamWConfig), C.c_int, C.POINTER(C.c_int64), C.POINTER(C.c_float), PP, PP,
+                               PP, PP, P]
+    lib.adamw_step.restype = C.c_int
     lib.muon_profile_enable.argtypes = [C.c_int]
     lib.muon_profile_enable.restype = None
     lib.muon_profile_read.argtypes = [C.POINTER(MuonProfileEntry), C.c_int]
@@ -295,3 +307,26 @@ def profile_read() -> dict:
         raise MuonError(MUON_ERR_CUDA, "muon_profile_read")
     return {arr[i].name.decode(): {"launches": int(arr[i].launches), "ms": arr[i].ms, "flops": arr[i].flops,
                                    "bytes": arr[i].bytes} for i in range(n)}
+
+
+def adamw_step(params: List, grads: List, exp_avg: List, exp_avg_sq: List, step: int, lr=0.01,
+               beta1: float = 0.8, beta2: float = 0.95, eps: float = 1e-10, weight_decay: float = 0.0,
+               stream=None, check: bool = True) -> int:
+    """Fused AdamW over tensors (any shape, contiguous).  `lr` is a float or a
+    per-tensor sequence.  Params/grads bf16 or fp32 (all alike); states fp32."""
+    n = len(params)
+    cfg = AdamWConfig()
+    load().adamw_config_default(C.byref(cfg))
+    per_tensor = not isinstance(lr, (int, float))
+    cfg.lr = 0.0 if per_tensor else float(lr)
+    cfg.beta1, cfg.beta2, cfg.eps, cfg.weight_decay, cfg.step = beta1, beta2, eps, weight_decay, int(step)
+    if n:
+        cfg.param_dtype = dtype_code(params[0])
+        cfg.grad_dtype = dtype_code(grads[0])
+    numels = (C.c_int64 * max(1, n))(*[int(p.numel()) for p in params])
+    lrs = (C.c_float * max(1, n))(*[float(x) for x in lr]) if per_tensor else None
+    code = load().adamw_step(C.byref(cfg), n, numels, lrs, _ptrs(params, n), _ptrs(grads, n), _ptrs(exp_avg, n),
+                             _ptrs(exp_avg_sq, n), _stream(stream))
+    if check:
+        _raise(code, "adamw_step")
+    return code

@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama_aurora", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--workload", default="llama_aurora", choices=sorted(WL.WORKLOADS) + ["llama_aux"])
     ap.add_argument("--layers", type=int, default=28, help="layers of the 3.8B set (28 = full)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -55,7 +55,13 @@ def parse():
     return ap.parse_args()
 
 
+AUX_WORKLOADS = {"llama_aux": WL.llama_3p8b_aux}
+AUX_METRIC = "AdamW auxiliary-parameter steps/s on the 3.8B non-matrix set (GB/s, % of HBM)"
+
+
 def make_workload(args):
+    if args.workload in AUX_WORKLOADS:
+        return AUX_WORKLOADS[args.workload](layers=args.layers)
     if args.workload in ("llama_plain", "llama_aurora"):
         return WL.WORKLOADS[args.workload](layers=args.layers)
     return WL.WORKLOADS[args.workload]()
@@ -209,6 +215,116 @@ def run_reference(args):
     return 0
 
 
+# --------------------------------------------------------------------------- AdamW leg
+AUX_BYTES_PER_ELEM = {("bf16", "bf16"): 2 + 2 + 2 + 8 + 8, ("f32", "f32"): 4 + 4 + 4 + 8 + 8}
+
+
+def aux_oracle_time(wl, idx):
+    import oracle.muon_oracle as O
+    P = [WL.aux_param(wl, i) for i in idx]
+    G = [WL.aux_grad(wl, i, 1) for i in idx]
+    t0 = time.perf_counter()
+    for k, i in enumerate(idx):
+        z = np.zeros(wl.shapes[i])
+        O.adamw_step(WL.to_f64(P[k], wl.param_dtype), WL.to_f64(G[k], wl.grad_dtype), z, z, wl.lrs[i], wl.beta1,
+                     wl.beta2, wl.eps, wl.weight_decay, 1)
+    return time.perf_counter() - t0
+
+
+def aux_cpu_line(wl, reps):
+    idx = [2] + list(range(16, min(wl.n, 24)))          # one value-embedding table and some 1-D tensors
+    elems = sum(int(np.prod(wl.shapes[i])) for i in idx)
+    ts = [aux_oracle_time(wl, idx) for _ in range(reps)]
+    step_s = sum(ts) / len(ts) * wl.elements() / elems
+    return 1.0 / step_s, {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                          "sample": f"{len(idx)} of {wl.n} tensors ({elems / 1e6:.1f} M elements) stepped by the "
+                                    f"float64 NumPy oracle, scaled by element count (x{wl.elements() / elems:.1f})"}
+
+
+def run_aux(args, wl):
+    import torch
+    from aurora_orthogonalised_optimizer_b200 import _abi as A
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        raise SystemExit("the AdamW workload runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pdt = torch.bfloat16 if wl.param_dtype == WL.BF16 else torch.float32
+
+    def dev_tensor(a, dt):
+        if dt == WL.BF16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    p = [dev_tensor(WL.aux_param(wl, i), wl.param_dtype) for i in range(wl.n)]
+    g = [dev_tensor(WL.aux_grad(wl, i, 1), wl.grad_dtype) for i in range(wl.n)]
+    m = [torch.zeros(s, dtype=torch.float32, device=dev) for s in wl.shapes]
+    v = [torch.zeros(s, dtype=torch.float32, device=dev) for s in wl.shapes]
+    stream = torch.cuda.current_stream(dev)
+    step_no = [0]
+
+    def step():
+        step_no[0] += 1
+        A.adamw_step(p, g, m, v, step_no[0], wl.lrs, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = "0"
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    launches_per_step = (wl.n + 191) // 192
+    bytes_step = wl.elements() * AUX_BYTES_PER_ELEM[(wl.param_dtype, wl.grad_dtype)]
+    peaks, kind = load_peaks()
+    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    gbs = bytes_step / ms / 1e6
+    e2e = None
+    if not args.no_e2e:
+        g_pin = [t.cpu().pin_memory() for t in g]
+        p_pin = [torch.empty_like(t, device="cpu").pin_memory() for t in p]
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            for k in range(wl.n):
+                g[k].copy_(g_pin[k], non_blocking=True)
+            step()
+            for k in range(wl.n):
+                p_pin[k].copy_(p[k], non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e = {"value": 1e3 * args.steps / f0.elapsed_time(f1), "unit": "steps/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in g_pin),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in p_pin)}
+    cpu = None
+    if not args.no_cpu_baseline:
+        _, cpu = aux_cpu_line(wl, 1)
+    line = {
+        "metric": AUX_METRIC, "value": 1e3 / ms, "unit": "steps/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0, 0.02^2) params, N(0, 1e-6) grads)",
+        "config": {"workload": wl.name, "tensors": wl.n, "elements": wl.elements(),
+                   "l2": "inputs (>20 GB) larger than the 126 MB L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "traffic": None, "kernel": "k_adamw", "peak_kind": f"hbm_gbs ({kind})",
+                     "bytes_per_launch": bytes_step / launches_per_step},
+        "gpu_launches": launches_per_step * args.steps, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------------- GPU leg
 def traffic_record(kernel_src):
     """Per-launch DRAM traffic from the committed ncu summary, if taken on this exact kernel source."""
@@ -227,6 +343,23 @@ def traffic_record(kernel_src):
 
 def main():
     args = parse()
+    if args.workload in AUX_WORKLOADS:
+        if args.impl == "reference":
+            if int(os.environ.get("RANK", "0")) != 0:
+                return 0
+            wl = make_workload(args)
+            for _ in range(args.warmup):
+                aux_cpu_line(wl, 1)
+            v, cpu = aux_cpu_line(wl, args.steps)
+            print(json.dumps({"impl": "reference", "metric": AUX_METRIC, "value": v, "unit": "steps/s",
+                              "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "strong",
+                              "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                              "config": {"workload": wl.name}, "cpu_baseline": cpu,
+                              "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+            return 0
+        return run_aux(args, make_workload(args))
     if args.impl == "reference":
         return run_reference(args)
 

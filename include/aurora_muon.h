@@ -169,6 +169,40 @@ muon_status uw_floor_apply(const muon_config* cfg, int n, const muon_shape* shap
                            const void* const* params, float* const* updates,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Auxiliary AdamW for the parameters Muon does not step (the Track 3
+ * write-up, "完整的超参配置表" and the hyper-parameter placement paragraph:
+ * token embedding lr 0.3, output projection lr 1/320, 1-D parameters lr 0.01,
+ * betas (0.8, 0.95), eps 1e-10, weight_decay 0, fused).  The pages name the
+ * optimizer without printing its update; this is torch.optim.AdamW's
+ * decoupled-weight-decay Adam at 1-based step count `step`:
+ *   p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+ *   p <- p - lr / (1 - b1^step) * m / (sqrt(v) / sqrt(1 - b2^step) + eps).
+ * adamw_config_default() fills lr 0.01, betas (0.8, 0.95), eps 1e-10, wd 0,
+ * step 1, bf16 params and grads. */
+typedef struct {
+  float lr;            /* used for every tensor when `lrs` is NULL */
+  float beta1, beta2;  /* in [0, 1) */
+  float eps;           /* >= 0 */
+  float weight_decay;  /* >= 0 (decoupled) */
+  int   step;          /* 1-based step count for the bias corrections */
+  int   param_dtype;   /* muon_dtype of params */
+  int   grad_dtype;    /* muon_dtype of grads */
+} adamw_config;
+
+void adamw_config_default(adamw_config* cfg);
+
+/* One fused AdamW step over n contiguous tensors of any shape.
+ * numels    : host array of n element counts (0 = skip the tensor).
+ * lrs       : host array of n learning rates, or NULL (cfg->lr for all).
+ * params    : n device pointers (param_dtype), updated in place.
+ * grads     : n device pointers (grad_dtype), read only.
+ * exp_avg, exp_avg_sq : n device pointers (fp32), updated in place.
+ * Every device pointer must be 16-byte aligned.  No workspace.  Errors:
+ * INVALID_ARG (before any launch), CUDA. */
+muon_status adamw_step(const adamw_config* cfg, int n, const int64_t* numels, const float* lrs,
+                       void* const* params, const void* const* grads, float* const* exp_avg,
+                       float* const* exp_avg_sq, void* stream);
+
 /* Synchronises `stream`, then returns and clears the sticky device status
  * word of the current device (MUON_OK, or MUON_ERR_TIMEOUT after a bounded
  * device wait gave up). */

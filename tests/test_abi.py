@@ -134,3 +134,25 @@ def test_other_entry_points_validate(lib):
     assert lib.uw_floor_apply(None, 1, sh, x, y, None, 0, None) == A.MUON_ERR_INVALID_ARG
     assert lib.uw_floor_apply(C.byref(cfg), 1, sh, x, _arr(None), None, 0, None) == A.MUON_ERR_INVALID_ARG
     assert lib.uw_floor_apply(C.byref(cfg), 1, sh, x, y, None, 0, None) == A.MUON_ERR_WORKSPACE
+
+
+def test_adamw_defaults_and_validation(lib):
+    c = A.AdamWConfig()
+    lib.adamw_config_default(C.byref(c))
+    assert c.beta1 == pytest.approx(0.8) and c.beta2 == pytest.approx(0.95)
+    assert c.eps == pytest.approx(1e-10) and c.weight_decay == 0.0 and c.step == 1
+    n1 = (C.c_int64 * 1)(16)
+    x = _arr(FAKE)
+    def call(cfg, numels=n1, p=x, g=x, m=x, v=x):
+        return lib.adamw_step(C.byref(cfg) if cfg is not None else None, 1, numels, None, p, g, m, v, None)
+    assert call(None) == A.MUON_ERR_INVALID_ARG
+    for field, bad in [("step", 0), ("beta1", 1.0), ("beta2", -0.1), ("eps", -1.0), ("weight_decay", -1.0),
+                       ("param_dtype", 3)]:
+        b = A.AdamWConfig()
+        lib.adamw_config_default(C.byref(b))
+        setattr(b, field, bad)
+        assert call(b) == A.MUON_ERR_INVALID_ARG, field
+    assert call(c, numels=(C.c_int64 * 1)(-1)) == A.MUON_ERR_INVALID_ARG
+    assert call(c, m=_arr(FAKE + 4)) == A.MUON_ERR_INVALID_ARG          # misaligned
+    assert call(c, g=_arr(None)) == A.MUON_ERR_INVALID_ARG
+    assert lib.adamw_step(C.byref(c), 0, None, None, None, None, None, None, None) == A.MUON_OK

@@ -288,3 +288,54 @@ def generate_torch(wl: Workload, indices: Optional[Sequence[int]] = None, step: 
     with ThreadPoolExecutor(max(1, threads)) as ex:
         res = list(ex.map(one, idx))
     return [r[0] for r in res], [r[1] for r in res]
+
+
+# --------------------------------------------------------------------------
+# the parameters the auxiliary AdamW steps (not the 2-D block matrices)
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class AuxWorkload:
+    name: str
+    seed: int
+    shapes: List[Tuple[int, ...]]
+    lrs: List[float]
+    param_dtype: str = BF16
+    grad_dtype: str = BF16
+    beta1: float = 0.8
+    beta2: float = 0.95
+    eps: float = 1e-10
+    weight_decay: float = 0.0
+
+    @property
+    def n(self) -> int:
+        return len(self.shapes)
+
+    def elements(self) -> int:
+        return sum(int(np.prod(s)) for s in self.shapes)
+
+
+def llama_3p8b_aux(layers: int = 28, vocab: int = 50304, d: int = 3072, kv: int = 1024,
+                   value_tables: int = 14) -> AuxWorkload:
+    """Token embedding (154.5M), untied LM head (154.5M), 14 value-embedding
+    tables (721.2M) and per-layer 1-D gains of the 3.8B model; lrs as the
+    Track 3 write-up sets them (embeddings 0.3, output projection 1/320,
+    1-D parameters 0.01)."""
+    shapes, lrs = [(vocab, d), (vocab, d)], [0.3, 1.0 / 320.0]
+    shapes += [(vocab, kv)] * value_tables
+    lrs += [0.3] * value_tables
+    for _ in range(layers):
+        shapes += [(d,), (d,), (1,), (1,)]       # two RMSNorm gains, two residual scalars
+        lrs += [0.01] * 4
+    return AuxWorkload("llama_3p8b_adamw_aux", 5, shapes, lrs)
+
+
+def aux_param(wl: AuxWorkload, idx: int) -> np.ndarray:
+    x = _rng(wl.seed, idx, 0, STREAM_W).standard_normal(wl.shapes[idx], dtype=np.float32)
+    x *= np.float32(0.02)
+    return store(x, wl.param_dtype)
+
+
+def aux_grad(wl: AuxWorkload, idx: int, step: int = 0) -> np.ndarray:
+    x = _rng(wl.seed, idx, step, STREAM_G).standard_normal(wl.shapes[idx], dtype=np.float32)
+    x *= np.float32(1e-3)
+    return store(x, wl.grad_dtype)
