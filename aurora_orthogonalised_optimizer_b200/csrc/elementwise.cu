@@ -139,22 +139,23 @@ __global__ void k_finalize_sums(const MatTable t, const double* partials, int nq
 //   mode 0 (D init):  D_j = 1 / max(sqrt(sum), pp_eps)              ["源码实现"]
 //   mode 1 (D update): row_sq = max(sum, pp_eps^2);
 //                      D_j *= (target / row_sq)^beta, target = s / l
-// A block owns 64 columns: 8 column groups of 8 x 32 row lanes, 16-byte loads.
+// A block owns kColStrip = 256 columns; each warp streams every 8th row with
+// one 16-byte load (8 columns) per lane, so a warp reads 512 contiguous bytes.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
-  __shared__ float part[32][kTile + 1];
+  __shared__ float part[kWarps][kColStrip];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
-  const int cg = threadIdx.x & 7, rl = threadIdx.x >> 3;
-  const int64_t j = (int64_t)b * kTile + 8 * cg;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t j = (int64_t)b * kColStrip + 8 * lane;
   const void* X = mode == 0 ? d.uX : d.UX;
   const bool vec = (d.ldl & 7) == 0;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (j < d.l) {
 #pragma unroll 4
-    for (int64_t i = rl; i < d.s; i += 32) {
+    for (int64_t i = w; i < d.s; i += kWarps) {
       float x[8];
       ld8r(X, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
 #pragma unroll
@@ -162,20 +163,19 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) part[rl][8 * cg + e] = acc[e];
+  for (int e = 0; e < 8; ++e) part[w][8 * lane + e] = acc[e];
   __syncthreads();
-  if (threadIdx.x < kTile) {
-    const int64_t jj = (int64_t)b * kTile + threadIdx.x;
-    if (jj < d.l) {
-      float sum = 0.f;
-      for (int r = 0; r < 32; ++r) sum += part[r][threadIdx.x];
-      if (mode == 0) {
-        d.D[jj] = 1.f / fmaxf(sqrtf(sum), pp_eps);
-      } else {
-        const float row_sq = fmaxf(sum, pp_eps * pp_eps);
-        const float target = (float)d.s / (float)d.l;
-        d.D[jj] = d.D[jj] * powf(target / row_sq, beta);
-      }
+  const int64_t jj = (int64_t)b * kColStrip + threadIdx.x;
+  if (jj < d.l) {
+    float sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < kWarps; ++r) sum += part[r][threadIdx.x];
+    if (mode == 0) {
+      d.D[jj] = 1.f / fmaxf(sqrtf(sum), pp_eps);
+    } else {
+      const float row_sq = fmaxf(sum, pp_eps * pp_eps);
+      const float target = (float)d.s / (float)d.l;
+      d.D[jj] = d.D[jj] * powf(target / row_sq, beta);
     }
   }
 }
@@ -278,13 +278,13 @@ __global__ void k_scalars(const MatTable t, int op, int src_slot, float ns_eps, 
 //   flag 0 (row dot):  out_i = sum_j Q_ij x_j   (x length l, out length s)
 //                      one warp per kMatvecRowsPerWarp rows, 8-element groups per lane
 //   flag 1 (col dot):  out_j = sum_i Q_ij y_i   (y length s, out length l)
-//                      64 columns per block, 8 groups x 32 row lanes
+//                      kColStrip columns per block, warps over rows
 // `dir` selects vec0 -> vec1 (0) or vec1 -> vec0 (1).  The vectors are
 // 16-byte aligned with length padded to a multiple of 64.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_matvec(const MatTable t, int dir) {
-  __shared__ float part[32][kTile + 1];
+  __shared__ float part[kWarps][kColStrip];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
@@ -319,12 +319,12 @@ k_matvec(const MatTable t, int dir) {
       }
     }
   } else {
-    const int cg = threadIdx.x & 7, rl = threadIdx.x >> 3;
-    const int64_t j = (int64_t)b * kTile + 8 * cg;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t j = (int64_t)b * kColStrip + 8 * lane;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (j < d.l) {
 #pragma unroll 4
-      for (int64_t i = rl; i < d.s; i += 32) {
+      for (int64_t i = w; i < d.s; i += kWarps) {
         float x[8];
         ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
         const float y = in[i];
@@ -333,15 +333,14 @@ k_matvec(const MatTable t, int dir) {
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[rl][8 * cg + e] = acc[e];
+    for (int e = 0; e < 8; ++e) part[w][8 * lane + e] = acc[e];
     __syncthreads();
-    if (threadIdx.x < kTile) {
-      const int64_t jj = (int64_t)b * kTile + threadIdx.x;
-      if (jj < d.l) {
-        float sum = 0.f;
-        for (int r = 0; r < 32; ++r) sum += part[r][threadIdx.x];
-        out[jj] = sum;
-      }
+    const int64_t jj = (int64_t)b * kColStrip + threadIdx.x;
+    if (jj < d.l) {
+      float sum = 0.f;
+#pragma unroll
+      for (int r = 0; r < kWarps; ++r) sum += part[r][threadIdx.x];
+      out[jj] = sum;
     }
   }
 }
@@ -490,6 +489,161 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
 }
 
 // ============================================================================
+// Flat streaming variants for matrices whose rows are contiguous and a
+// multiple of 8 elements long (no transposition needed): a block walks
+// kEwTilesPerCta chunks of kFlatChunk consecutive elements, each thread
+// moving two 8-element groups per chunk with 16-byte accesses.  Partials:
+// one slot per chunk, like the tiled kernels' one slot per tile.
+// ============================================================================
+__global__ void __launch_bounds__(kEwThreads)
+k_prologue_flat(const MatTable t, int mode, float mu, int nesterov, int want_w2, double* partials) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t total = d.m * d.n;
+  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int64_t c = c0; c < c0 + kEwTilesPerCta && c * kFlatChunk < total; ++c) {
+    float su2 = 0.f, sw2 = 0.f;
+    float g[2][8], m[2][8], w[2][8];
+    bool in[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+      in[k] = e < total;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) g[k][q] = m[k][q] = w[k][q] = 0.f;
+      if (!in[k]) continue;
+      ld8(d.G, e, t.grad_dtype, g[k]);
+      if (mode == 0) {
+        ld8(d.M, e, kF32, m[k]);
+        if (want_w2) ld8(d.W, e, t.param_dtype, w[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!in[k]) continue;
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+      float u[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (mode == 0) {
+          m[k][q] = m[k][q] + (1.f - mu) * (g[k][q] - m[k][q]);
+          u[q] = nesterov ? g[k][q] + mu * (m[k][q] - g[k][q]) : m[k][q];
+        } else {
+          u[q] = g[k][q];
+        }
+        su2 += u[q] * u[q];
+        sw2 += w[k][q] * w[k][q];
+      }
+      if (mode == 0) st8(d.M, e, kF32, m[k]);
+      st8(d.uX, e, t.ns_dtype, u);
+    }
+    warp_partials(partials, d.part + c, 2, su2, sw2);
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads)
+k_scale_cols_flat(const MatTable t, double* partials) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t total = d.s * d.l;
+  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int64_t c = c0; c < c0 + kEwTilesPerCta && c * kFlatChunk < total; ++c) {
+    float s2 = 0.f;
+    float x[2][8], dj[2][8];
+    bool in[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+      in[k] = e < total;
+      if (!in[k]) continue;
+      ld8(d.uX, e, t.ns_dtype, x[k]);
+      ld8(d.D, e % d.l, kF32, dj[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!in[k]) continue;
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        x[k][q] *= dj[k][q];
+        s2 += x[k][q] * x[k][q];
+      }
+      st8(d.X0, e, t.ns_dtype, x[k]);
+    }
+    warp_partials(partials, d.part + c, 1, s2, 0.f);
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads)
+k_dots_flat(const MatTable t, double* partials) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t total = d.s * d.l;
+  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int64_t c = c0; c < c0 + kEwTilesPerCta && c * kFlatChunk < total; ++c) {
+    float a = 0.f, cc = 0.f;
+    float U[2][8], u[2][8];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) U[k][q] = u[k][q] = 0.f;
+      if (e < total) {
+        ld8(d.UX, e, t.ns_dtype, U[k]);
+        ld8(d.uX, e, t.ns_dtype, u[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        a += U[k][q] * U[k][q];
+        cc += U[k][q] * u[k][q];
+      }
+    warp_partials(partials, d.part + c, 2, a, cc);
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads)
+k_epilogue_flat(const MatTable t, float lr, int update_w, const double* scal) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t total = d.m * d.n;
+  const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
+  const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
+  const bool need_U = cU != 0.f, need_u = cu != 0.f;
+  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  for (int64_t c = c0; c < c0 + kEwTilesPerCta && c * kFlatChunk < total; ++c) {
+    float U[2][8], u[2][8], w[2][8];
+    bool in[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+      in[k] = e < total;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) U[k][q] = u[k][q] = w[k][q] = 0.f;
+      if (!in[k]) continue;
+      if (need_U) ld8(d.UX, e, t.ns_dtype, U[k]);
+      if (need_u) ld8(d.uX, e, t.ns_dtype, u[k]);
+      if (update_w) ld8(d.W, e, t.param_dtype, w[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!in[k]) continue;
+      const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[q] = cU * U[k][q] + cu * u[k][q];
+        w[k][q] -= lr * v[q];
+      }
+      if (d.V) st8(d.V, e, kF32, v);
+      if (update_w) st8(d.W, e, t.param_dtype, w[k]);
+    }
+  }
+}
+
+// ============================================================================
 // u/w floor on caller-provided fp32 updates (entry point uw_floor_apply):
 // partial |W|^2 and |V|^2 over the flat original layout (4096 elements per
 // block, 16-byte accesses), then V *= coef.
@@ -566,6 +720,28 @@ cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int 
                                  int slot1, double* scal, cudaStream_t st) {
   if (t.count == 0) return cudaSuccess;
   k_finalize_sums<<<t.count, 256, 0, st>>>(t, partials, nq, slot0, slot1, scal);
+  return cudaGetLastError();
+}
+cudaError_t launch_prologue_flat(const MatTable& t, int nblk, int mode, float mu, int nesterov, int want_w2,
+                                 double* partials, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_prologue_flat<<<nblk, kEwThreads, 0, st>>>(t, mode, mu, nesterov, want_w2, partials);
+  return cudaGetLastError();
+}
+cudaError_t launch_scale_cols_flat(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_scale_cols_flat<<<nblk, kEwThreads, 0, st>>>(t, partials);
+  return cudaGetLastError();
+}
+cudaError_t launch_dots_flat(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_dots_flat<<<nblk, kEwThreads, 0, st>>>(t, partials);
+  return cudaGetLastError();
+}
+cudaError_t launch_epilogue_flat(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
+                                 cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_epilogue_flat<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
   return cudaGetLastError();
 }
 cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, float beta,

@@ -304,6 +304,23 @@ int64_t tiles_x(const MatDesc& d) { return cdiv(d.s, 64) * cdiv(d.l, 64); }
 // blocks of a streaming launch (kEwTilesPerCta tiles each)
 int64_t blocks_orig(const MatDesc& d) { return cdiv(tiles_orig(d), kEwTilesPerCta); }
 int64_t blocks_x(const MatDesc& d) { return cdiv(tiles_x(d), kEwTilesPerCta); }
+// Flat streaming applies when rows are contiguous, a multiple of 8 long and
+// (original orientation) need no transposition into the X orientation.
+bool flat_orig(const MatDesc& d) { return !d.tall && (d.n & 7) == 0 && d.ldl == d.n; }
+bool flat_x(const MatDesc& d) { return (d.l & 7) == 0 && d.ldl == d.l; }
+int64_t fblocks_orig(const MatDesc& d) { return cdiv(cdiv(d.m * d.n, kFlatChunk), kEwTilesPerCta); }
+int64_t fblocks_x(const MatDesc& d) { return cdiv(cdiv(d.s * d.l, kFlatChunk), kEwTilesPerCta); }
+// partial-sum slots a stage leaves per matrix (one per tile or per flat chunk)
+int64_t slots_orig(const MatDesc& d) { return flat_orig(d) ? cdiv(d.m * d.n, kFlatChunk) : tiles_orig(d); }
+int64_t slots_x(const MatDesc& d) { return flat_x(d) ? cdiv(d.s * d.l, kFlatChunk) : tiles_x(d); }
+
+// Split ids by a predicate on their descriptors.
+template <class Pred>
+std::pair<std::vector<int>, std::vector<int>> split_ids(const Ctx& c, const std::vector<int>& ids, Pred pred) {
+  std::pair<std::vector<int>, std::vector<int>> r;
+  for (int i : ids) (pred(make_desc(c, i)) ? r.first : r.second).push_back(i);
+  return r;
+}
 
 #define CK(expr)                                   \
   do {                                             \
@@ -315,11 +332,16 @@ int64_t blocks_x(const MatDesc& d) { return cdiv(tiles_x(d), kEwTilesPerCta); }
 muon_status stage_prologue(const Ctx& c, const std::vector<int>& ids, int mode, bool want_w2) {
   const double per_elem = dt_bytes(c.grad_dtype) + c.plan->nsb + (mode == 0 ? 8.0 : 0.0) +
                           (want_w2 ? dt_bytes(c.param_dtype) : 0.0);
-  CK(for_chunks(c, ids, blocks_orig, [&](const MatTable& t, int nb) {
+  const auto fl = split_ids(c, ids, flat_orig);
+  CK(for_chunks(c, fl.first, fblocks_orig, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
+    return launch_prologue_flat(t, nb, mode, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
+  }));
+  CK(for_chunks(c, fl.second, blocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_prologue(t, nb, mode, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
   }));
-  CK(for_chunks(c, ids, tiles_orig, [&](const MatTable& t, int) {
+  CK(for_chunks(c, ids, slots_orig, [&](const MatTable& t, int) {
     ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
     return launch_finalize_sums(t, c.partials, 2, S_SUM_U2, want_w2 ? S_SUM_W2 : -1, c.scal, c.st);
   }));
@@ -343,7 +365,7 @@ muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int
     return for_chunks(c, ids, [first](MatDesc& d) -> int64_t {
       const bool rowdot = first ? !d.tall : (bool)d.tall;
       d.flag = rowdot ? 0 : 1;
-      return rowdot ? cdiv(d.s, kMatvecRowsPerCta) : cdiv(d.l, 64);
+      return rowdot ? cdiv(d.s, kMatvecRowsPerCta) : cdiv(d.l, kColStrip);
     }, [&](const MatTable& t, int nb) {
       ProfScope ps(PC_POWER, 2.0 * table_elems(t), c.plan->nsb * table_elems(t), c.st);
       return launch_matvec(t, nb, dir, c.st);
@@ -502,18 +524,23 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       return launch_copy_rho(t, c.scal, c.st);
     }));
   if (!eq_ids.empty())
-    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
+    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
       ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
       return launch_colnorm(t, nb, 0, pe, beta, c.st);
     }));
   const int rounds = eq_b.empty() ? 1 : c.cfg->pp_iterations;
   for (int k = 0; k < rounds; ++k) {
     if (!eq_ids.empty()) {
-      CK(for_chunks(c, eq_ids, blocks_x, [&](const MatTable& t, int nb) {
+      const auto fx = split_ids(c, eq_ids, flat_x);
+      CK(for_chunks(c, fx.first, fblocks_x, [&](const MatTable& t, int nb) {
+        ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
+        return launch_scale_cols_flat(t, nb, c.partials, c.st);
+      }));
+      CK(for_chunks(c, fx.second, blocks_x, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
         return launch_scale_cols(t, nb, c.partials, c.st);
       }));
-      CK(for_chunks(c, eq_ids, tiles_x, [&](const MatTable& t, int) {
+      CK(for_chunks(c, eq_ids, slots_x, [&](const MatTable& t, int) {
         ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
         cudaError_t e = launch_finalize_sums(t, c.partials, 1, S_SUM_X02, -1, c.scal, c.st);
         if (e != cudaSuccess) return e;
@@ -529,7 +556,7 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
     muon_status s = stage_newton_schulz(c, bids, in_q);
     if (s != MUON_OK) return s;
     if (k < rounds - 1)
-      CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, 64); }, [&](const MatTable& t, int nb) {
+      CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
         return launch_colnorm(t, nb, 1, pe, beta, c.st);
       }));
@@ -548,7 +575,12 @@ muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool updat
   const bool need_u = c.cfg->contra != 0.f || !update_w;
   const double per_elem = c.plan->nsb * (need_u ? 2.0 : 1.0) + (update_w ? 2.0 * dt_bytes(c.param_dtype) : 0.0) +
                           (c.V ? 4.0 : 0.0);
-  CK(for_chunks(c, ids, blocks_orig, [&](const MatTable& t, int nb) {
+  const auto fl = split_ids(c, ids, flat_orig);
+  CK(for_chunks(c, fl.first, fblocks_orig, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
+    return launch_epilogue_flat(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
+  }));
+  CK(for_chunks(c, fl.second, blocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_epilogue(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
   }));
@@ -556,11 +588,16 @@ muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool updat
 }
 
 muon_status stage_dots(const Ctx& c, const std::vector<int>& ids) {
-  CK(for_chunks(c, ids, blocks_x, [&](const MatTable& t, int nb) {
+  const auto fx = split_ids(c, ids, flat_x);
+  CK(for_chunks(c, fx.first, fblocks_x, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_REDUCE, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
+    return launch_dots_flat(t, nb, c.partials, c.st);
+  }));
+  CK(for_chunks(c, fx.second, blocks_x, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_REDUCE, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
     return launch_dots(t, nb, c.partials, c.st);
   }));
-  CK(for_chunks(c, ids, tiles_x, [&](const MatTable& t, int) {
+  CK(for_chunks(c, ids, slots_x, [&](const MatTable& t, int) {
     ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
     return launch_finalize_sums(t, c.partials, 2, S_SUM_UU2, S_DOT_UUX, c.scal, c.st);
   }));

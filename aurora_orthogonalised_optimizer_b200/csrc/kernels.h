@@ -58,9 +58,15 @@ cudaError_t read_and_clear_device_status(unsigned int* out);  // current device
 // consecutive tiles of one matrix (launch ceil(tiles / kEwTilesPerCta)
 // blocks per matrix); reductions still leave one set of partials per tile.
 constexpr int kEwTilesPerCta = 4;
+// Flat variants (rows contiguous, length a multiple of 8): chunks of
+// kFlatChunk elements, one partial slot per chunk.
+constexpr int64_t kFlatChunk = 4096;
 // Row-dot pass of the power iteration: 8 warps x kMatvecRowsPerWarp rows.
 constexpr int kMatvecRowsPerWarp = 4;
 constexpr int kMatvecRowsPerCta = 8 * kMatvecRowsPerWarp;
+// Column reductions (Aurora column norms, power-iteration column dots):
+// one block per kColStrip columns of the X orientation.
+constexpr int kColStrip = 256;
 cudaError_t launch_prologue(const MatTable& t, int nblk, int mode, float mu, int nesterov,
                             int want_w2, double* partials, cudaStream_t st);
 cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int nq, int slot0,
@@ -79,6 +85,12 @@ cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w,
 cudaError_t launch_sumsq_wv(const MatTable& t, int nblk, double* partials, cudaStream_t st);
 cudaError_t launch_scale_v(const MatTable& t, int nblk, const double* scal, cudaStream_t st);
 cudaError_t launch_copy_rho(const MatTable& t, const double* scal, cudaStream_t st);
+cudaError_t launch_prologue_flat(const MatTable& t, int nblk, int mode, float mu, int nesterov, int want_w2,
+                                 double* partials, cudaStream_t st);
+cudaError_t launch_scale_cols_flat(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+cudaError_t launch_dots_flat(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+cudaError_t launch_epilogue_flat(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
+                                 cudaStream_t st);
 cudaError_t launch_sigma_out(const MatTable& t, const double* scal, float* sigma_out, cudaStream_t st);
 
 }  // namespace am
