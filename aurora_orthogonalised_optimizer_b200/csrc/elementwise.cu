@@ -278,13 +278,13 @@ __global__ void k_scalars(const MatTable t, int op, int src_slot, float ns_eps, 
 //   flag 0 (row dot):  out_i = sum_j Q_ij x_j   (x length l, out length s)
 //                      one warp per kMatvecRowsPerWarp rows, 8-element groups per lane
 //   flag 1 (col dot):  out_j = sum_i Q_ij y_i   (y length s, out length l)
-//                      kColStrip columns per block, warps over rows
+//                      kColDotStrip columns per block, 32 row lanes
 // `dir` selects vec0 -> vec1 (0) or vec1 -> vec0 (1).  The vectors are
 // 16-byte aligned with length padded to a multiple of 64.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
 k_matvec(const MatTable t, int dir) {
-  __shared__ float part[kWarps][kColStrip];
+  __shared__ float smem[32 * (kColDotStrip + 1)];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
@@ -299,6 +299,7 @@ k_matvec(const MatTable t, int dir) {
 #pragma unroll
     for (int r = 0; r < kMatvecRowsPerWarp; ++r) acc[r] = 0.f;
     if (i0 < d.s) {
+#pragma unroll 2
       for (int64_t j = 8 * lane; j < d.l; j += 256) {
         float v[8];
         ld8r(in, 0, j, d.l, true, kF32, v);
@@ -319,12 +320,14 @@ k_matvec(const MatTable t, int dir) {
       }
     }
   } else {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int64_t j = (int64_t)b * kColStrip + 8 * lane;
+    // kColDotStrip = 64 columns: 8 groups of 8 columns x 32 row lanes
+    float (*part)[kColDotStrip + 1] = reinterpret_cast<float (*)[kColDotStrip + 1]>(smem);
+    const int cg = threadIdx.x & 7, rl = threadIdx.x >> 3;
+    const int64_t j = (int64_t)b * kColDotStrip + 8 * cg;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (j < d.l) {
 #pragma unroll 4
-      for (int64_t i = w; i < d.s; i += kWarps) {
+      for (int64_t i = rl; i < d.s; i += 32) {
         float x[8];
         ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
         const float y = in[i];
@@ -333,14 +336,15 @@ k_matvec(const MatTable t, int dir) {
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[w][8 * lane + e] = acc[e];
+    for (int e = 0; e < 8; ++e) part[rl][8 * cg + e] = acc[e];
     __syncthreads();
-    const int64_t jj = (int64_t)b * kColStrip + threadIdx.x;
-    if (jj < d.l) {
-      float sum = 0.f;
-#pragma unroll
-      for (int r = 0; r < kWarps; ++r) sum += part[r][threadIdx.x];
-      out[jj] = sum;
+    if (threadIdx.x < kColDotStrip) {
+      const int64_t jj = (int64_t)b * kColDotStrip + threadIdx.x;
+      if (jj < d.l) {
+        float sum = 0.f;
+        for (int r = 0; r < 32; ++r) sum += part[r][threadIdx.x];
+        out[jj] = sum;
+      }
     }
   }
 }
@@ -430,47 +434,54 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
     const bool need_U = cU != 0.f, need_u = cu != 0.f;
     const bool vec = (d.n & 7) == 0;
     const bool xvec = (d.ldl & 7) == 0;
-    if (d.tall) {
-      // X tile rows = original columns c0 + xr, X tile columns = original rows r0 + 8 cg ..
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int xr = rg + 32 * k;
-        const int64_t xi = c0 + xr, xj = r0 + 8 * cg;
-        float U[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (xi < d.n && xj < d.m) {
-          if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, U);
-          if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, u);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          tU[xr][8 * cg + e] = U[e];
-          tu[xr][8 * cg + e] = u[e];
-        }
-      }
-      __syncthreads();
-    }
     const int64_t j = c0 + 8 * cg;
     float U[2][8], u[2][8], w[2][8];
     bool in[2];
+    // parameter rows first: their loads overlap the transpose below
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int rr = rg + 32 * k;
-      const int64_t i = r0 + rr;
+      const int64_t i = r0 + rg + 32 * k;
       in[k] = i < d.m && j < d.n;
 #pragma unroll
       for (int e = 0; e < 8; ++e) U[k][e] = u[k][e] = w[k][e] = 0.f;
-      if (!in[k]) continue;
-      if (d.tall) {
+      if (in[k] && update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
+    }
+    if (d.tall) {
+      // X tile rows = original columns c0 + xr, X tile columns = original rows r0 + 8 cg ..
+      float xU[2][8], xu[2][8];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int64_t xi = c0 + rg + 32 * k, xj = r0 + 8 * cg;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xU[k][e] = xu[k][e] = 0.f;
+        if (xi < d.n && xj < d.m) {
+          if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xU[k]);
+          if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xu[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          U[k][e] = tU[8 * cg + e][rr];
-          u[k][e] = tu[8 * cg + e][rr];
+          tU[rg + 32 * k][8 * cg + e] = xU[k][e];
+          tu[rg + 32 * k][8 * cg + e] = xu[k][e];
         }
-      } else {
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          U[k][e] = tU[8 * cg + e][rg + 32 * k];
+          u[k][e] = tu[8 * cg + e][rg + 32 * k];
+        }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int64_t i = r0 + rg + 32 * k;
+        if (!in[k]) continue;
         if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U[k]);
         if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u[k]);
       }
-      if (update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {

@@ -365,7 +365,7 @@ muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int
     return for_chunks(c, ids, [first](MatDesc& d) -> int64_t {
       const bool rowdot = first ? !d.tall : (bool)d.tall;
       d.flag = rowdot ? 0 : 1;
-      return rowdot ? cdiv(d.s, kMatvecRowsPerCta) : cdiv(d.l, kColStrip);
+      return rowdot ? cdiv(d.s, kMatvecRowsPerCta) : cdiv(d.l, kColDotStrip);
     }, [&](const MatTable& t, int nb) {
       ProfScope ps(PC_POWER, 2.0 * table_elems(t), c.plan->nsb * table_elems(t), c.st);
       return launch_matvec(t, nb, dir, c.st);

@@ -67,6 +67,8 @@ constexpr int kMatvecRowsPerCta = 8 * kMatvecRowsPerWarp;
 // Column reductions (Aurora column norms, power-iteration column dots):
 // one block per kColStrip columns of the X orientation.
 constexpr int kColStrip = 256;
+// Power-iteration column dots: one block per kColDotStrip columns.
+constexpr int kColDotStrip = 64;
 cudaError_t launch_prologue(const MatTable& t, int nblk, int mode, float mu, int nesterov,
                             int want_w2, double* partials, cudaStream_t st);
 cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int nq, int slot0,

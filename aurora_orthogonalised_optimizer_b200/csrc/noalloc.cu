@@ -116,7 +116,7 @@ extern "C" muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, c
         MatDesc& d = t.mats[k];
         d.flag = pass == 2 ? 1 : 0;
         d.nblk = pass == 1 ? (int)((d.s + kMatvecRowsPerCta - 1) / kMatvecRowsPerCta)
-                 : pass == 2 ? (int)((d.l + kColStrip - 1) / kColStrip) : 0;
+                 : pass == 2 ? (int)((d.l + kColDotStrip - 1) / kColDotStrip) : 0;
         t.blk_prefix[k] = tot;
         tot += d.nblk;
       }
