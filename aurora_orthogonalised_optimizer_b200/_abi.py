@@ -24,7 +24,7 @@ MUON_GEMM_BF16, MUON_GEMM_FP32, MUON_GEMM_BF16_SIMT = 0, 1, 2
 EXPORTS = ["muon_config_default", "muon_workspace_size", "muon_step", "ns_polar", "aurora_polar",
            "opnorm_normalize", "uw_floor_apply", "muon_last_device_status", "muon_status_string",
            "muon_profile_enable", "muon_profile_read", "opnorm_normalize_noalloc",
-           "adamw_config_default", "adamw_step"]
+           "adamw_config_default", "adamw_step", "muon_selftest_wait_timeout"]
 
 
 class MuonShape(C.Structure):
@@ -94,6 +94,8 @@ def load():
     lib.uw_floor_apply.argtypes = [C.POINTER(MuonConfig), C.c_int, C.POINTER(MuonShape), PP, PP, P,
                                    C.c_size_t, P]
     lib.uw_floor_apply.restype = C.c_int
+    lib.muon_selftest_wait_timeout.argtypes = [C.c_longlong, P]
+    lib.muon_selftest_wait_timeout.restype = C.c_int
     lib.muon_last_device_status.argtypes = [P]
     lib.muon_last_device_status.restype = C.c_int
     lib.muon_status_string.argtypes = [C.c_int]
@@ -289,6 +291,11 @@ def uw_floor_apply(cfg: Config, params: List, updates: List, workspace=None, str
     if check:
         _raise(code, "uw_floor_apply")
     return code
+
+
+def selftest_wait_timeout(max_cycles: int = 1_000_000, stream=None) -> int:
+    """Run the bounded-wait timeout path once on the device (see the header)."""
+    return int(load().muon_selftest_wait_timeout(int(max_cycles), _stream(stream)))
 
 
 def last_device_status(stream=None) -> int:

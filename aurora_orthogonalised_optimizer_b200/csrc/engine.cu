@@ -825,6 +825,11 @@ int muon_profile_read(muon_profile_entry* out, int max_entries) {
   return w;
 }
 
+muon_status muon_selftest_wait_timeout(long long max_cycles, void* stream) {
+  const long long lim = std::min(std::max(max_cycles, 1000LL), 4000000000LL);
+  return launch_wait_selftest(lim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
+
 muon_status muon_last_device_status(void* stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
   unsigned int v = 0;

@@ -100,14 +100,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
 }
 // Bounded wait; returns false (and raises the abort flag) on timeout or when
 // another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 255u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         raise_status(MUON_ERR_TIMEOUT);
         return false;
@@ -611,6 +612,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   }
 }
 
+// Exercises the timeout path of mbar_wait: one thread waits on a barrier
+// that nothing ever arrives on; after `limit` cycles the wait gives up and
+// records MUON_ERR_TIMEOUT.
+__global__ void k_wait_selftest(long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, limit);
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -685,6 +701,11 @@ DeviceFacts device_facts(int num_sms) {
 }
 
 }  // namespace
+
+cudaError_t launch_wait_selftest(long long limit_cycles, cudaStream_t st) {
+  k_wait_selftest<<<1, 32, 0, st>>>(limit_cycles);
+  return cudaGetLastError();
+}
 
 cudaError_t read_and_clear_device_status(unsigned int* out) {
   unsigned int v = 0, zero = 0;

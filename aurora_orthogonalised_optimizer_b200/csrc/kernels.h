@@ -52,6 +52,7 @@ cudaError_t launch_gemm_tc(const GemmLaunch& L, const void* maps, int num_sms, b
 bool tc_encode_maps(const GemmLaunch& L, bool pair, void* maps_out);  // host: builds the tensor maps
 int tc_tile_count(int kind, int M, int N, bool pair, int* tiles_m, int* tiles_n);
 cudaError_t read_and_clear_device_status(unsigned int* out);  // current device
+cudaError_t launch_wait_selftest(long long limit_cycles, cudaStream_t st);
 
 // ---------------------------------------------------------------- element-wise
 // Streaming kernels work on 64 x 64 tiles; a block walks kEwTilesPerCta

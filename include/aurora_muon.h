@@ -208,6 +208,16 @@ muon_status adamw_step(const adamw_config* cfg, int n, const int64_t* numels, co
  * device wait gave up). */
 muon_status muon_last_device_status(void* stream);
 
+/* Diagnostic of the failure-detection path (no counterpart on the pages):
+ * launches one block whose thread waits, with the same bounded-wait routine
+ * the GEMM kernels use, on a shared-memory barrier that nothing arrives on.
+ * After max_cycles SM clock cycles (clamped to [1e3, 4e9]) the wait gives
+ * up and records MUON_ERR_TIMEOUT in the sticky device status word, exactly
+ * as a stalled pipeline would; the kernel then returns and the context stays
+ * usable.  Returns MUON_OK when the launch succeeded (read the outcome with
+ * muon_last_device_status), MUON_ERR_CUDA otherwise. */
+muon_status muon_selftest_wait_timeout(long long max_cycles, void* stream);
+
 /* Static English description of a status code. */
 const char* muon_status_string(muon_status s);
 
