@@ -156,3 +156,11 @@ def test_adamw_defaults_and_validation(lib):
     assert call(c, m=_arr(FAKE + 4)) == A.MUON_ERR_INVALID_ARG          # misaligned
     assert call(c, g=_arr(None)) == A.MUON_ERR_INVALID_ARG
     assert lib.adamw_step(C.byref(c), 0, None, None, None, None, None, None, None) == A.MUON_OK
+
+
+def test_size_limits_are_rejected_on_the_host(lib):
+    p, g, m = _arr(FAKE), _arr(FAKE + 4096), _arr(FAKE + 8192)
+    # the smaller side above 32768 is not supported; nothing is sized or launched
+    assert _call_step(lib, _cfg(), [(40000, 40000)], p, g, m) == A.MUON_ERR_UNSUPPORTED
+    assert A.workspace_size(A.Config(), [(40000, 40000)]) == 0
+    assert _call_step(lib, _cfg(), [(1 << 32, 8)], p, g, m) == A.MUON_ERR_INVALID_ARG

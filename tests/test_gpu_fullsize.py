@@ -74,3 +74,45 @@ def test_llama_3p8b_aurora_stack_full_size():
 def test_llama_3p8b_plain_muon_full_size():
     wl = WL.llama_3p8b_plain()
     _run(wl, [1, 6 * 27 + 2])
+
+
+def _run_sampled_trajectory(wl, sample, gemm_mode=A.MUON_GEMM_BF16, tol=3e-2):
+    """All matrices of the workload stepped together (one call per step, as the
+    bench does); the sampled ones follow the oracle's own trajectory."""
+    pdt = A.MUON_BF16 if wl.param_dtype == WL.BF16 else A.MUON_F32
+    gdt = A.MUON_BF16 if wl.grad_dtype == WL.BF16 else A.MUON_F32
+    cfg = A.Config.from_step_config(wl.cfg, gemm_mode=gemm_mode, param_dtype=pdt, grad_dtype=gdt)
+    W, _ = WL.generate_torch(wl, None, 0, threads=16, want_g=False)
+    p = [w.cuda() for w in W]
+    m = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    v = [torch.empty(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    ws = A.make_workspace(cfg, wl.shapes)
+    Wn, _, _ = WL.generate(wl, sample)
+    oW = {k: WL.to_f64(Wn[j], wl.param_dtype) for j, k in enumerate(sample)}
+    oM = {k: np.zeros(wl.shapes[k]) for k in sample}
+    for st in range(wl.steps):
+        _, G = WL.generate_torch(wl, None, st, threads=16, want_w=False)
+        g = [x.cuda() for x in G]
+        A.muon_step(cfg, p, g, m, v, ws)
+        torch.cuda.synchronize()
+        assert A.last_device_status() == A.MUON_OK
+        for k in sample:
+            gk = WL.to_f64(WL.grad(wl, k, st), wl.grad_dtype)
+            oW[k], oM[k], V = O.step(oW[k], gk, oM[k], wl.cfg, wl.param_dtype)
+            ev = rel_fro(f64(v[k]), V)
+            assert ev <= tol, ("V", st, k, wl.shapes[k], ev)
+            assert rel_fro(f64(m[k]), oM[k]) <= 1e-6, ("m", st, k)
+
+
+def test_gpt2_124m_all_72_matrices_five_steps():
+    """GPT-2 124M set, plain Muon, mu 0.90, lr 0.04: all 72 matrices per call,
+    5 steps; layers 0 and 11 against the oracle at every step."""
+    wl = WL.gpt2_124m_plain()
+    _run_sampled_trajectory(wl, list(range(6)) + list(range(66, 72)))
+
+
+def test_aurora_sweep_all_128_matrices():
+    """Aurora sweep (32 each of 1024x4096, 4096x1024, 2048^2, 768x3072), full
+    stack, fp32 params/grads: all 128 per call, one of each shape sampled."""
+    wl = WL.aurora_shape_sweep()
+    _run_sampled_trajectory(wl, [5, 37, 69, 101])

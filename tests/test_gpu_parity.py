@@ -259,3 +259,12 @@ def test_grads_not_mutated():
     A.muon_step(cfg, p, g, m, None, A.make_workspace(cfg, shapes))
     torch.cuda.synchronize()
     assert torch.equal(g[0], g0)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+def test_step_more_shape_buckets_than_one_gemm_launch_holds(mode):
+    """20 distinct shapes: more buckets than one grouped GEMM launch carries,
+    so every Newton-Schulz GEMM is split over several launches."""
+    shapes = [(16 + 8 * i, 24 + 4 * i) if i % 2 else (40 + 4 * i, 16 + 8 * i) for i in range(20)]
+    wl = WL.custom("many_buckets", 11, shapes, WL.aurora_stack(), WL.BF16, WL.BF16, w_std=0.05)
+    run_steps(wl, MODES[mode])
