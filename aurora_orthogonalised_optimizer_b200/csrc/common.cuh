@@ -121,12 +121,14 @@ struct MatDesc {
   float* vec0;        // power-iteration vectors (length >= l), two of them
   float* vec1;
   float* rho_slot;    // bucket-ordered copy of rho read by the GEMM epilogues
+  float* gvp;         // fused power iteration: one partial X^T z (ldl floats) per row item
   int64_t m, n, s, l, ldl;
   int tall;           // m > n
   int idx;            // matrix index (scalar block row)
   int part;           // first partial slot of this matrix
   int nblk;           // blocks of this matrix in the current launch
   int flag;           // launch-specific per-matrix flag
+  int gv_rows;        // fused power iteration: rows of X per item
 };
 
 constexpr int kMaxMatsPerLaunch = 96;

@@ -34,6 +34,8 @@ struct MatPlan {
   int64_t m, n, s, l;
   int tall, bucket, bidx;
   int64_t part;      // first partial block slot
+  int64_t gv_rows;   // fused power iteration: rows of X per item
+  int64_t gv_off;    // and the offset (floats) of this matrix's item partials
 };
 
 struct BucketPlan {
@@ -47,8 +49,17 @@ struct Plan {
   int nsb = 2;
   std::vector<MatPlan> mats;
   std::vector<BucketPlan> buckets;
-  size_t off_scal = 0, off_partials = 0, total = 0;
+  size_t off_scal = 0, off_partials = 0, off_gv = 0, total = 0;
 };
+
+// Rows per item of the fused power-iteration pass: items of about
+// total / (148 x 8) elements (a few waves of one block per SM), kept between
+// 64 Ki and 1 Mi elements; the partial X^T z per item then costs at most
+// ~2% of the item's bytes.
+int64_t gv_rows_for(int64_t s, int64_t l, int64_t total_elems) {
+  const int64_t item = std::min<int64_t>(std::max<int64_t>(total_elems / (148 * 8), 1 << 16), 1 << 20);
+  return std::max<int64_t>(1, std::min<int64_t>(s, cdiv(item, l)));
+}
 
 int ns_dtype_of(const muon_config* c) { return c->gemm_mode == MUON_GEMM_FP32 ? kF32 : kBF16; }
 
@@ -57,7 +68,8 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
   p.ns_dtype = ns_dtype_of(cfg);
   p.nsb = dt_bytes(p.ns_dtype);
   std::map<std::pair<int64_t, int64_t>, int> bmap;
-  int64_t part = 0;
+  int64_t part = 0, gv = 0, total_elems = 0;
+  for (int i = 0; i < n; ++i) total_elems += shapes[i].rows * shapes[i].cols;
   for (int i = 0; i < n; ++i) {
     MatPlan mp;
     mp.m = shapes[i].rows;
@@ -82,6 +94,9 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
     mp.part = part;
     const int64_t tiles = cdiv(mp.m, 64) * cdiv(mp.n, 64);
     part += std::max(tiles, cdiv(mp.m * mp.n, 4096));
+    mp.gv_rows = gv_rows_for(mp.s, mp.l, total_elems);
+    mp.gv_off = gv;
+    gv += cdiv(mp.s, mp.gv_rows) * round8(mp.l);
     p.mats.push_back(mp);
   }
   size_t off = 0;
@@ -104,6 +119,8 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
   off = align_up(off + (size_t)n * S_COUNT * sizeof(double));
   p.off_partials = off;
   off = align_up(off + (size_t)part * 8 /*warps*/ * 2 * sizeof(double));
+  p.off_gv = off;
+  off = align_up(off + (size_t)gv * sizeof(float));
   p.total = off;
   return p;
 }
@@ -258,6 +275,8 @@ MatDesc make_desc(const Ctx& c, int i) {
   d.vec0 = wsp<float>(c, b.off_v0) + vo;
   d.vec1 = wsp<float>(c, b.off_v1) + vo;
   d.rho_slot = wsp<float>(c, b.off_rho) + mp.bidx;
+  d.gvp = wsp<float>(c, c.plan->off_gv) + mp.gv_off;
+  d.gv_rows = (int)mp.gv_rows;
   d.m = mp.m; d.n = mp.n; d.s = mp.s; d.l = mp.l; d.ldl = b.ldl;
   d.tall = mp.tall;
   d.idx = i;
@@ -353,7 +372,9 @@ muon_status stage_prologue(const Ctx& c, const std::vector<int>& ids, int mode, 
 // Wide/square (X = A): t is a row dot of X, w a column dot.
 // Tall (X = A^T):      t is a column dot of X, w a row dot.
 // k_matvec flag: 0 = row dot (in: l, out: s), 1 = column dot (in: s, out: l).
-muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int iters) {
+// Separate row-dot and column-dot passes: two reads of X per iteration.  Used
+// for rows longer than the fused pass takes.
+muon_status stage_power_iteration_2pass(const Ctx& c, const std::vector<int>& ids, int iters) {
   auto vec_blocks = [](MatDesc& d) -> int64_t { d.flag = d.tall ? 1 : 0; return 0; };
   auto vecop = [&](int which, int mode, int len_is_s_when_flag0) {
     return for_chunks(c, ids, vec_blocks, [&](const MatTable& t, int) {
@@ -379,6 +400,57 @@ muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int
   }
   CK(pass(true, 0));           // t = A v
   CK(vecop(1, 2, 1));          // sigma = |t|
+  return MUON_OK;
+}
+
+// Fused passes (powiter.cu): one read of X per iteration, six in all.
+//   wide (v over l in vec0):   [z = X v -> vec1, vec0 = X^T z / |X^T z|] x iters;
+//                              z = X v -> vec1; sigma = |vec1| (over s).
+//   tall (v over s in vec0):   vec1 = X^T v0 (= A v0);
+//                              [z = X vec1 -> vec0, vec1 = X^T z / |z|] x iters;
+//                              sigma = |vec1| (over l).
+muon_status stage_power_iteration(const Ctx& c, const std::vector<int>& ids, int iters) {
+  const int64_t max_ldl = gv_max_ldl(c.plan->ns_dtype);
+  const auto fz = split_ids(c, ids, [max_ldl](const MatDesc& d) { return d.ldl <= max_ldl; });
+  if (!fz.second.empty()) {
+    muon_status s = stage_power_iteration_2pass(c, fz.second, iters);
+    if (s != MUON_OK) return s;
+  }
+  const std::vector<int>& all = fz.first;
+  if (all.empty()) return MUON_OK;
+  const auto tw = split_ids(c, all, [](const MatDesc& d) { return d.tall != 0; });
+  auto vec_blocks = [](MatDesc& d) -> int64_t { d.flag = d.tall ? 1 : 0; return 0; };
+  auto items = [](MatDesc& d) -> int64_t { d.flag = d.tall ? 1 : 0; return cdiv(d.s, d.gv_rows); };
+  auto pass = [&](const std::vector<int>& v, int mode) {
+    return for_chunks(c, v, items, [&](const MatTable& t, int nb) {
+      const double fl = (mode == GV_DOT_ACC ? 4.0 : 2.0) * table_elems(t);
+      ProfScope ps(PC_POWER, fl, c.plan->nsb * table_elems(t), c.st);
+      return launch_gramvec(t, nb, mode, c.st);
+    });
+  };
+  auto reduce = [&](const std::vector<int>& v, int normalise) {
+    return for_chunks(c, v, vec_blocks, [&](const MatTable& t, int) {
+      ProfScope ps(PC_POWER, 0.0, 0.0, c.st);
+      return launch_gv_reduce(t, normalise, c.st);
+    });
+  };
+  auto vecop = [&](int which, int mode, int len_is_s_when_flag0) {
+    return for_chunks(c, all, vec_blocks, [&](const MatTable& t, int) {
+      ProfScope ps(PC_POWER, 0.0, 0.0, c.st);
+      return launch_vecop(t, which, mode, len_is_s_when_flag0, c.scal, c.st);
+    });
+  };
+  CK(vecop(0, 0, 0));                                   // v0 = 1/sqrt(len) (wide: l, tall: s)
+  if (!tw.first.empty()) {
+    CK(pass(tw.first, GV_ACC));                         // tall: X^T v0
+    CK(reduce(tw.first, 0));
+  }
+  for (int k = 0; k < iters; ++k) {
+    CK(pass(all, GV_DOT_ACC));
+    CK(reduce(all, 1));
+  }
+  if (!tw.second.empty()) CK(pass(tw.second, GV_DOT));  // wide: z = X v
+  CK(vecop(1, 2, 1));                                   // sigma = |vec1|
   return MUON_OK;
 }
 
@@ -832,9 +904,10 @@ muon_status muon_selftest_wait_timeout(long long max_cycles, void* stream) {
 
 muon_status muon_last_device_status(void* stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
-  unsigned int v = 0;
+  unsigned int v = 0, w = 0;
   if (read_and_clear_device_status(&v) != cudaSuccess) return MUON_ERR_CUDA;
-  return static_cast<muon_status>(v);
+  if (read_and_clear_gv_status(&w) != cudaSuccess) return MUON_ERR_CUDA;
+  return static_cast<muon_status>(v != 0 ? v : w);
 }
 
 }  // extern "C"

@@ -94,6 +94,16 @@ cudaError_t launch_scale_cols_flat(const MatTable& t, int nblk, double* partials
 cudaError_t launch_dots_flat(const MatTable& t, int nblk, double* partials, cudaStream_t st);
 cudaError_t launch_epilogue_flat(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
                                  cudaStream_t st);
+// Fused power-iteration pass (powiter.cu): one read of X (s x l) per pass.
+enum GramVecMode {
+  GV_DOT_ACC = 0,   // z = X y (written), partial X^T z
+  GV_DOT = 1,       // z = X y only
+  GV_ACC = 2        // partial X^T z with z given
+};
+int64_t gv_max_ldl(int ns_dtype);   // longest row (elements, padded) the fused pass takes
+cudaError_t launch_gramvec(const MatTable& t, int nblk, int mode, cudaStream_t st);
+cudaError_t launch_gv_reduce(const MatTable& t, int normalise, cudaStream_t st);
+cudaError_t read_and_clear_gv_status(unsigned int* out);
 cudaError_t launch_sigma_out(const MatTable& t, const double* scal, float* sigma_out, cudaStream_t st);
 
 }  // namespace am

@@ -122,6 +122,31 @@ def test_opnorm_normalize_matches_oracle(mode):
         assert rel_fro(f64(outs[i]), N) <= tol
 
 
+@pytest.mark.parametrize("mode", ["fp32", "bf16"])
+def test_opnorm_fused_pass_team_widths_items_and_fallback(mode):
+    """The power iteration reads each row of the s x l orientation once per
+    iteration when l (padded to 8) is at most 12288 (bf16 staging) or 8192
+    (fp32), with 1 to 16 warps per row; longer rows take the two-pass path.
+    Shapes cover every team width, rows split over several items, ragged l,
+    both orientations, and the first length past each limit."""
+    cfg = A.Config(gemm_mode=MODES[mode])
+    shapes = [(300, 1000), (5, 2040), (4000, 7), (2000, 300), (3, 8190), (8192, 2), (8200, 2), (2, 8201)]
+    if mode == "bf16":
+        shapes += [(2, 12288), (12290, 3)]
+    mats = [gauss(s, 700 + i) for i, s in enumerate(shapes)]
+    ins = [torch.from_numpy(m).cuda() for m in mats]
+    outs = [torch.empty(m.shape, dtype=torch.float32, device="cuda") for m in mats]
+    sig = torch.zeros(len(mats), dtype=torch.float32, device="cuda")
+    A.opnorm_normalize(cfg, ins, outs, sig, A.make_workspace(cfg, shapes))
+    torch.cuda.synchronize()
+    assert A.last_device_status() == A.MUON_OK
+    tol = 1e-5 if mode == "fp32" else 1e-2
+    for i, m in enumerate(mats):
+        N, s = O.scale_to_unit_operator_norm(m.astype(np.float64), 5)
+        assert abs(sig[i].item() - s) <= tol * s, (m.shape, sig[i].item(), s)
+        assert rel_fro(f64(outs[i]), N) <= tol, m.shape
+
+
 # ------------------------------------------------------------------ u/w floor
 def test_uw_floor_apply_matches_oracle():
     shapes = [(64, 32), (100, 300), (7, 9)]
