@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", default="bf16", choices=["bf16", "fp32", "bf16simt"])
+    ap.add_argument("--ns-vs-cublas", action="store_true",
+                    help="time one Newton-Schulz polar of the workload's matrices on this library (ns_polar) "
+                         "and the same iteration on torch/cuBLAS bf16 bmm, alternating; prints one JSON line")
     return ap.parse_args()
 
 
@@ -326,6 +329,82 @@ def run_aux(args, wl):
 
 
 # --------------------------------------------------------------------------- GPU leg
+def run_ns_vs_cublas(args):
+    """Context measurement: the same Newton-Schulz polar (ns_steps x {A = X X^T,
+    B = b A + c A^2, X = a X + B X} over every matrix of the workload, bf16
+    operands) through ns_polar and through torch.bmm/baddbmm on cuBLAS, in
+    alternating rounds on the same GPU with clocks sampled.  FLOPs are counted
+    the library's way (one triangle of each symmetric product) for both."""
+    import torch
+    from aurora_orthogonalised_optimizer_b200 import _abi as A
+    wl = make_workload(args)
+    dev = torch.cuda.current_device()
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    c = wl.cfg
+    buckets = {}
+    for m, n in wl.shapes:
+        key = (min(m, n), max(m, n))
+        buckets[key] = buckets.get(key, 0) + 1
+    useful = sum(cnt * c.ns_steps * (l * s * (s + 1) + s * s * (s + 1) + 2.0 * s * s * l)
+                 for (s, l), cnt in buckets.items())
+    g = torch.Generator(device="cuda").manual_seed(0)
+    X = {k: torch.randn(cnt, k[0], k[1], device="cuda", dtype=torch.bfloat16, generator=g) / (k[0] * k[1]) ** 0.5
+         for k, cnt in buckets.items()}
+    ins = [torch.randn(m, n, device="cuda", dtype=torch.bfloat16, generator=g) for m, n in wl.shapes]
+    outs = [torch.empty(m, n, device="cuda", dtype=torch.float32) for m, n in wl.shapes]
+    cfg = A.Config.from_step_config(c, gemm_mode=A.MUON_GEMM_BF16)
+    ws = A.make_workspace(cfg, wl.shapes)
+
+    def cublas_polar():
+        for x in X.values():
+            for _ in range(c.ns_steps):
+                a = torch.bmm(x, x.transpose(1, 2))
+                b = torch.baddbmm(a, a, a, beta=c.ns_b, alpha=c.ns_c)
+                x = torch.baddbmm(x, b, x, beta=c.ns_a, alpha=1.0)
+
+    def ours():
+        A.ns_polar(cfg, ins, outs, ws)
+
+    def timed(fn, reps):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    for _ in range(max(1, args.warmup)):
+        ours()
+        cublas_polar()
+    rows = {"library_ns_polar": [], "cublas_bmm": []}
+    for _ in range(max(1, args.steps)):
+        for name, fn in (("library_ns_polar", ours), ("cublas_bmm", cublas_polar)):
+            cs = ClockSampler(gpu_id)
+            cs.start()
+            if name == "library_ns_polar":
+                A.profile_enable(True)
+            ms = timed(fn, 3)
+            row = {"ms_per_polar": ms, "useful_tflops": useful / ms / 1e9}
+            if name == "library_ns_polar":
+                prof = A.profile_read()
+                A.profile_enable(False)
+                gm = prof.get("ns_gemm_tc")
+                if gm:
+                    row["gemm_ms_per_polar"] = gm["ms"] / 3
+                    row["gemm_useful_tflops"] = gm["flops"] / gm["ms"] / 1e9
+            row["clocks"] = cs.stop()
+            rows[name].append(row)
+    best = {k: min(v, key=lambda r: r["ms_per_polar"]) for k, v in rows.items()}
+    print(json.dumps({"metric": "Newton-Schulz polar of the workload's matrices, library vs torch/cuBLAS",
+                      "workload": wl.name, "ns_steps": c.ns_steps, "useful_gflop_per_polar": useful / 1e9,
+                      "library": best["library_ns_polar"], "cublas": best["cublas_bmm"],
+                      "speedup": best["cublas_bmm"]["ms_per_polar"] / best["library_ns_polar"]["ms_per_polar"],
+                      "rounds": rows}), flush=True)
+    return 0
+
+
 def traffic_record(kernel_src):
     """Per-launch DRAM traffic from the committed ncu summary, if taken on this exact kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -343,6 +422,8 @@ def traffic_record(kernel_src):
 
 def main():
     args = parse()
+    if args.ns_vs_cublas:
+        return run_ns_vs_cublas(args)
     if args.workload in AUX_WORKLOADS:
         if args.impl == "reference":
             if int(os.environ.get("RANK", "0")) != 0:
