@@ -418,24 +418,23 @@ k_dots(const MatTable t, double* partials) {
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads, 4)
 k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
-  __shared__ float tU[kTile][kTile + 1];
-  __shared__ float tu[kTile][kTile + 1];
+  __shared__ float tV[kTile][kTile + 1];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int nt = (int)(((d.m + kTile - 1) / kTile) * ((d.n + kTile - 1) / kTile));
   const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
+  const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
+  const bool need_U = cU != 0.f, need_u = cu != 0.f;
+  const bool vec = (d.n & 7) == 0;
+  const bool xvec = (d.ldl & 7) == 0;
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
   for (int b = b0; b < b0 + kEwTilesPerCta && b < nt; ++b) {
     if (b != b0) __syncthreads();   // shared tile reused by the next tile
     const int64_t tiles_c = (d.n + kTile - 1) / kTile;
     const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
-    const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
-    const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
-    const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
-    const bool need_U = cU != 0.f, need_u = cu != 0.f;
-    const bool vec = (d.n & 7) == 0;
-    const bool xvec = (d.ldl & 7) == 0;
     const int64_t j = c0 + 8 * cg;
-    float U[2][8], u[2][8], w[2][8];
+    float v[2][8], w[2][8];
     bool in[2];
     // parameter rows first: their loads overlap the transpose below
 #pragma unroll
@@ -443,57 +442,52 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
       const int64_t i = r0 + rg + 32 * k;
       in[k] = i < d.m && j < d.n;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) U[k][e] = u[k][e] = w[k][e] = 0.f;
+      for (int e = 0; e < 8; ++e) v[k][e] = w[k][e] = 0.f;
       if (in[k] && update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
     }
     if (d.tall) {
-      // X tile rows = original columns c0 + xr, X tile columns = original rows r0 + 8 cg ..
-      float xU[2][8], xu[2][8];
+      // V = cU U + cu u is formed in the X orientation (X tile rows = original
+      // columns c0 + xr, X tile columns = original rows r0 + 8 cg ..) and
+      // transposed through one shared tile
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int64_t xi = c0 + rg + 32 * k, xj = r0 + 8 * cg;
+        float xU[8], xu[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) xU[k][e] = xu[k][e] = 0.f;
+        for (int e = 0; e < 8; ++e) xU[e] = xu[e] = 0.f;
         if (xi < d.n && xj < d.m) {
-          if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xU[k]);
-          if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xu[k]);
+          if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xU);
+          if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xu);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tV[rg + 32 * k][8 * cg + e] = cU * xU[e] + cu * xu[e];
       }
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          tU[rg + 32 * k][8 * cg + e] = xU[k][e];
-          tu[rg + 32 * k][8 * cg + e] = xu[k][e];
-        }
       __syncthreads();
 #pragma unroll
       for (int k = 0; k < 2; ++k)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          U[k][e] = tU[8 * cg + e][rg + 32 * k];
-          u[k][e] = tu[8 * cg + e][rg + 32 * k];
-        }
+        for (int e = 0; e < 8; ++e) v[k][e] = tV[8 * cg + e][rg + 32 * k];
     } else {
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int64_t i = r0 + rg + 32 * k;
         if (!in[k]) continue;
-        if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U[k]);
-        if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u[k]);
+        float U[8], u[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) U[e] = u[e] = 0.f;
+        if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U);
+        if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[k][e] = cU * U[e] + cu * u[e];
       }
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       if (!in[k]) continue;
       const int64_t ro = (r0 + rg + 32 * k) * d.n;
-      float v[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[e] = cU * U[k][e] + cu * u[k][e];
-        w[k][e] -= lr * v[e];
-      }
-      if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v);
+      for (int e = 0; e < 8; ++e) w[k][e] -= lr * v[k][e];
+      if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v[k]);
       if (update_w) st8r(d.W, ro, j, d.n, vec, t.param_dtype, w[k]);
     }
   }

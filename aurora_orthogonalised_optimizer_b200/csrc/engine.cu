@@ -195,9 +195,15 @@ bool tc_pair() {
 }
 
 // ---------------------------------------------------------------- tracing
-enum ProfClass { PC_GEMM_TC = 0, PC_GEMM_SIMT, PC_PROLOGUE, PC_POWER, PC_AURORA, PC_REDUCE, PC_EPILOGUE, PC_COUNT };
+// The tc_kind_* classes time the same tensor-core launches as ns_gemm_tc,
+// split by GEMM kind (Gram, square, update); they are not extra launches.
+enum ProfClass {
+  PC_GEMM_TC = 0, PC_GEMM_SIMT, PC_PROLOGUE, PC_POWER, PC_AURORA, PC_REDUCE, PC_EPILOGUE,
+  PC_TC_GRAM, PC_TC_SQR, PC_TC_UPD, PC_COUNT
+};
 const char* const kProfNames[PC_COUNT] = {"ns_gemm_tc", "ns_gemm_simt", "prologue", "power_iter",
-                                          "aurora_rows", "reductions", "epilogue"};
+                                          "aurora_rows", "reductions", "epilogue",
+                                          "tc_kind_gram", "tc_kind_square", "tc_kind_update"};
 
 struct ProfRecord {
   int cls;
@@ -472,6 +478,7 @@ muon_status gemm_launch(const Ctx& c, GemmLaunch& L) {
     alignas(64) unsigned char maps[kMaxGemmGroups * 3 * 128];
     if (!tc_encode_maps(L, tc_pair(), maps)) return MUON_ERR_CUDA;
     ProfScope ps(PC_GEMM_TC, gemm_flops(L), 0.0, c.st);
+    ProfScope pk(PC_TC_GRAM + L.g[0].kind, gemm_flops(L), 0.0, c.st);   // every group of a launch has one kind
     CK(launch_gemm_tc(L, maps, num_sms_current(), tc_pair(), c.st));
   } else {
     ProfScope ps(PC_GEMM_SIMT, gemm_flops(L), 0.0, c.st);

@@ -575,6 +575,8 @@ def main():
     peaks, peak_kind = load_peaks()
     gk = "ns_gemm_tc" if gemm == A.MUON_GEMM_BF16 else "ns_gemm_simt"
     g = prof.get(gk, {"launches": 0, "ms": 0.0, "flops": 0.0})
+    kinds = {k[len("tc_kind_"):]: v for k, v in prof.items() if k.startswith("tc_kind_")}
+    prof = {k: v for k, v in prof.items() if not k.startswith("tc_kind_")}
     launches = sum(v["launches"] for v in prof.values())
     achieved_tf = g["flops"] / max(g["ms"], 1e-9) / 1e9  # flops / ms -> TFLOP/s
     peak_tf = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
@@ -601,6 +603,11 @@ def main():
         if v["flops"] > 0:
             st["TFLOP/s"] = v["flops"] / v["ms"] / 1e9
         stages[k] = st
+    if gk in stages and kinds:
+        # the tensor-core GEMM launches split by kind (Gram, square, update)
+        stages[gk]["kinds"] = {k: {"launches": v["launches"] // args.steps, "ms_per_step": v["ms"] / args.steps,
+                                   "TFLOP/s": v["flops"] / max(v["ms"], 1e-9) / 1e9}
+                               for k, v in kinds.items() if v["launches"]}
     ns_nominal = nominal_ns_flops(wl)
     ns_tf_nominal = ns_nominal * steps_per_s / 1e12
 
