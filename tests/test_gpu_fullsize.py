@@ -3,8 +3,9 @@ in the launch configuration the bench times: one muon_step call over every
 matrix, tensor-core Newton-Schulz.
 
 * Sampled outputs: the k and v matrices (1024 x 3072) of the first and the
-  last layer are recomputed by the float64 oracle; update V within 3e-2
-  relative Frobenius error, momentum within 1e-6.
+  last layer, and (second Aurora test) one fc (12288 x 3072), one proj
+  (3072 x 12288) and one q (3072 x 3072), are recomputed by the float64
+  oracle; update V within 3e-2 relative Frobenius error, momentum within 1e-6.
 * Properties that hold for every matrix at any size, checked on all 168:
   - first step from zero momentum: m = (1 - mu) g up to fp32 rounding;
   - the parameter add: W_new = W - lr V up to the bf16 rounding of W_new
@@ -69,6 +70,14 @@ def test_llama_3p8b_aurora_stack_full_size():
     wl = WL.llama_3p8b_aurora()
     # k, v of layer 0 and of layer 27 (1024 x 3072, the Aurora wide path)
     _run(wl, [1, 2, 6 * 27 + 1, 6 * 27 + 2])
+
+
+def test_llama_3p8b_aurora_stack_full_size_tall_wide_square():
+    wl = WL.llama_3p8b_aurora()
+    # fc of layer 0 (12288 x 3072: tall, transposed into the X orientation,
+    # two Aurora polars), proj of layer 13 (3072 x 12288: wide, two polars)
+    # and q of layer 27 (3072 x 3072: square, one polar)
+    _run(wl, [4, 6 * 13 + 5, 6 * 27])
 
 
 def test_llama_3p8b_plain_muon_full_size():
