@@ -42,6 +42,8 @@ struct BucketPlan {
   int64_t s, l, ldl, lds;
   std::vector<int> members;
   size_t off_uX, off_P, off_Q, off_A, off_B, off_D, off_v0, off_v1, off_rho;
+  size_t off_dots;       // fused <U,U>, <U,u> partials of the last update GEMM (16 doubles per tile)
+  int64_t dot_tiles;     // tiles per member reserved there (both tensor-core variants fit)
 };
 
 struct Plan {
@@ -49,7 +51,7 @@ struct Plan {
   int nsb = 2;
   std::vector<MatPlan> mats;
   std::vector<BucketPlan> buckets;
-  size_t off_scal = 0, off_partials = 0, off_gv = 0, total = 0;
+  size_t off_scal = 0, off_partials = 0, off_gv = 0, off_dots = 0, total = 0;
 };
 
 // Rows per item of the fused power-iteration pass: items of about
@@ -114,6 +116,17 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
     b.off_v0 = off; off = align_up(off + vbytes);
     b.off_v1 = off; off = align_up(off + vbytes);
     b.off_rho = off; off = align_up(off + cnt * 4);
+  }
+  // per-tile reduction slots of the fused dots (tensor-core mode only)
+  p.off_dots = off;
+  for (auto& b : p.buckets) {
+    int tm, tn;
+    b.dot_tiles = 0;
+    if (cfg->gemm_mode == MUON_GEMM_BF16)
+      b.dot_tiles = std::max(tc_tile_count(GK_UPD, (int)b.s, (int)b.l, true, &tm, &tn),
+                             tc_tile_count(GK_UPD, (int)b.s, (int)b.l, false, &tm, &tn));
+    b.off_dots = off;
+    off = align_up(off + b.members.size() * (size_t)b.dot_tiles * 16 * sizeof(double));
   }
   p.off_scal = off;
   off = align_up(off + (size_t)n * S_COUNT * sizeof(double));
@@ -258,6 +271,7 @@ struct Ctx {
   float* const* M;
   float* const* V;
   int param_dtype, grad_dtype;
+  bool fuse_dots;    // the last update GEMM of each bucket's final polar forms <U,U>, <U,u>
 };
 
 template <class T> T* wsp(const Ctx& c, size_t off) { return reinterpret_cast<T*>(c.ws + off); }
@@ -507,7 +521,7 @@ void add_group(const Ctx& c, GemmLaunch& L, GemmGroup g) {
 // x0_in_Q (Aurora's D-scaled input); the iterates ping-pong P (even it),
 // Q (odd it).
 muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids_in,
-                                const std::vector<bool>& x0_in_Q_in) {
+                                const std::vector<bool>& x0_in_Q_in, const std::vector<bool>& final_in) {
   const Plan& p = *c.plan;
   const float a = c.cfg->ns_a, bc = c.cfg->ns_b, cc = c.cfg->ns_c;
   // Longest tiles first: the persistent kernel deals tiles round-robin in
@@ -520,11 +534,13 @@ muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids
     return bx.s != by.s ? bx.s > by.s : bx.l > by.l;
   });
   std::vector<int> bucket_ids;
-  std::vector<bool> x0_in_Q;
+  std::vector<bool> x0_in_Q, final_polar;
   for (size_t k : order) {
     bucket_ids.push_back(bucket_ids_in[k]);
     x0_in_Q.push_back(x0_in_Q_in[k]);
+    final_polar.push_back(final_in[k]);
   }
+  const bool tc = c.cfg->gemm_mode == MUON_GEMM_BF16;
   for (int it = 0; it < c.cfg->ns_steps; ++it) {
     for (int kind = 0; kind < 3; ++kind) {
       GemmLaunch L;
@@ -563,6 +579,10 @@ muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids
           g.E = X_in; g.lde = b.ldl; g.se = sx;
           g.alpha0 = 1.f; g.beta0 = a;
           g.pa = g.pb = it == 0 ? 1 : 0;
+          if (tc && c.fuse_dots && final_polar[k] && it == c.cfg->ns_steps - 1) {
+            g.dotu = c.ws + b.off_uX;
+            g.dotp = wsp<double>(c, b.off_dots);
+          }
         }
         add_group(c, L, g);
         if (L.num_groups == kMaxGemmGroups) {
@@ -629,10 +649,10 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       }));
     }
     std::vector<int> bids = eq_b;
-    std::vector<bool> in_q(eq_b.size(), true);
+    std::vector<bool> in_q(eq_b.size(), true), fin(eq_b.size(), k == rounds - 1);
     if (k == 0)
-      for (int b : plain_b) { bids.push_back(b); in_q.push_back(false); }
-    muon_status s = stage_newton_schulz(c, bids, in_q);
+      for (int b : plain_b) { bids.push_back(b); in_q.push_back(false); fin.push_back(true); }
+    muon_status s = stage_newton_schulz(c, bids, in_q, fin);
     if (s != MUON_OK) return s;
     if (k < rounds - 1)
       CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
@@ -679,6 +699,24 @@ muon_status stage_dots(const Ctx& c, const std::vector<int>& ids) {
   CK(for_chunks(c, ids, slots_x, [&](const MatTable& t, int) {
     ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
     return launch_finalize_sums(t, c.partials, 2, S_SUM_UU2, S_DOT_UUX, c.scal, c.st);
+  }));
+  return MUON_OK;
+}
+
+// <U,U> and <U,u> from the slots the last update GEMM of the final polar
+// filled (tensor-core mode): one block of 8 warp slots per output tile.
+muon_status stage_dots_fused(const Ctx& c, const std::vector<int>& ids) {
+  const Plan& p = *c.plan;
+  const bool pair = tc_pair();
+  CK(for_chunks(c, ids, [&](MatDesc& d) -> int64_t {
+    const BucketPlan& b = p.buckets[p.mats[d.idx].bucket];
+    int tm, tn;
+    const int64_t tpm = tc_tile_count(GK_UPD, (int)b.s, (int)b.l, pair, &tm, &tn);
+    d.part = (int)((b.off_dots - p.off_dots) / (16 * sizeof(double)) + (size_t)p.mats[d.idx].bidx * tpm);
+    return tpm;
+  }, [&](const MatTable& t, int) {
+    ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
+    return launch_finalize_sums(t, wsp<double>(c, p.off_dots), 2, S_SUM_UU2, S_DOT_UUX, c.scal, c.st);
   }));
   return MUON_OK;
 }
@@ -781,8 +819,9 @@ muon_status muon_step(const muon_config* cfg, int n, const muon_shape* shapes, v
   const std::vector<int> ids = iota_ids(n);
   if ((s = stage_prologue(c, ids, 0, cfg->target_uw > 0.f)) != MUON_OK) return s;
   if (cfg->contra != 0.f && (s = stage_power_iteration(c, ids, cfg->power_iters)) != MUON_OK) return s;
+  c.fuse_dots = cfg->gemm_mode == MUON_GEMM_BF16;
   if ((s = stage_polar(c, cfg->aurora != 0)) != MUON_OK) return s;
-  if ((s = stage_dots(c, ids)) != MUON_OK) return s;
+  if ((s = c.fuse_dots ? stage_dots_fused(c, ids) : stage_dots(c, ids)) != MUON_OK) return s;
   if ((s = set_coeffs(c, ids, 1)) != MUON_OK) return s;
   return stage_epilogue(c, ids, true, cfg->lr);
 }

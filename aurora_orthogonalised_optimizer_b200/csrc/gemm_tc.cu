@@ -530,17 +530,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         const int c0 = ti.n0 + ch * 32;
         return r0 < G.M && c0 < G.N && !(sym && c0 < r0);
       };
-      uint4 en[4] = {};
+      // fused reductions of the output against itself and against dotu
+      const bool dots = G.dotp != nullptr;
+      const __nv_bfloat16* Urow =
+          (dots && row < G.M) ? reinterpret_cast<const __nv_bfloat16*>(G.dotu) + (int64_t)ti.b * G.sc +
+                                    (int64_t)row * G.ldc
+                              : nullptr;
+      float s_cc = 0.f, s_cu = 0.f;
+      uint4 en[4] = {}, un[4] = {};
       int next = 0;
       while (next < TBN / 32 && !wanted(next)) ++next;
       if (next < TBN / 32 && Erow) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
+      if (next < TBN / 32 && Urow) load_e_chunk(Urow, ti.n0 + next * 32, G.N, un);
       while (next < TBN / 32) {
         const int ch = next;
         const int col0 = ti.n0 + ch * 32;
         const uint4 ec[4] = {en[0], en[1], en[2], en[3]};
+        const uint4 uc[4] = {un[0], un[1], un[2], un[3]};
         ++next;
         while (next < TBN / 32 && !wanted(next)) ++next;
         if (next < TBN / 32 && Erow) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
+        if (next < TBN / 32 && Urow) load_e_chunk(Urow, ti.n0 + next * 32, G.N, un);
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN + ch * 32), r);
         uint32_t pk[16];
@@ -556,6 +566,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             }
             const __nv_bfloat162 p2 = __floats2bfloat162_rn(v0, v1);
             pk[h] = *reinterpret_cast<const uint32_t*>(&p2);
+          }
+        }
+        if (Urow) {
+          // columns past N hold 0 in both (zero-filled operands and addend)
+          const uint32_t uw[16] = {uc[0].x, uc[0].y, uc[0].z, uc[0].w, uc[1].x, uc[1].y, uc[1].z, uc[1].w,
+                                   uc[2].x, uc[2].y, uc[2].z, uc[2].w, uc[3].x, uc[3].y, uc[3].z, uc[3].w};
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            const float v0 = bf16_bits_to_f(pk[h] & 0xFFFFu), v1 = bf16_bits_to_f(pk[h] >> 16);
+            s_cc = fmaf(v0, v0, fmaf(v1, v1, s_cc));
+            s_cu = fmaf(v0, bf16_bits_to_f(uw[h] & 0xFFFFu), fmaf(v1, bf16_bits_to_f(uw[h] >> 16), s_cu));
           }
         }
         // staging buffers of this parity are free once the group issued two
@@ -589,6 +610,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           bulk_commit();
         }
         par ^= 1u;
+      }
+      if (dots) {
+        // one slot per (tile, epilogue warp of the pair); unused slots of the
+        // single-SM variant are written as zero
+        s_cc = warp_sum(s_cc);
+        s_cu = warp_sum(s_cu);
+        if (lane == 0) {
+          const int tin = ti.m0 / Gm::kTileM + G.tiles_m * (ti.n0 / TBN);
+          double* slot = G.dotp + ((int64_t)ti.b * G.tiles_per_mat + tin) * 16;
+          const int w = (int)rank * 4 + q;
+          slot[2 * w] = (double)s_cc;
+          slot[2 * w + 1] = (double)s_cu;
+          if (!PAIR) {
+            slot[2 * (w + 4)] = 0.0;
+            slot[2 * (w + 4) + 1] = 0.0;
+          }
+        }
       }
       // this warp's TMEM reads of the accumulator are complete: release it
       tc_fence_before();

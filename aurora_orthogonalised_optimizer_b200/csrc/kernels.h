@@ -31,6 +31,12 @@ struct GemmGroup {
   const float* rho;               // per-batch normalisation scale (may be null)
   float alpha0, beta0;            // alpha = alpha0 * rho^pa, beta = beta0 * rho^pb
   int pa, pb;
+  // Update kind, tensor-core path only: when dotp is set the epilogue also
+  // forms per-warp partials of <C, C> and <C, dotu> (dotu laid out like C,
+  // bf16) over the stored bf16 values:
+  // dotp[((b * tiles_per_mat + tile) * 8 + warp) * 2 + {0, 1}].
+  const void* dotu;
+  double* dotp;
 };
 
 constexpr int kMaxGemmGroups = 16;
