@@ -26,7 +26,7 @@ constexpr int kAwThreads = 256;
 constexpr int kAwMaxTensors = 192;
 // A block owns kAwThreads * 8 * ITERS consecutive elements of one tensor.
 template <int ITERS>
-constexpr int64_t aw_chunk() { return (int64_t)kAwThreads * 8 * ITERS; }
+__host__ __device__ constexpr int64_t aw_chunk() { return (int64_t)kAwThreads * 8 * ITERS; }
 
 struct AwTensor {
   void* p;

@@ -123,24 +123,23 @@ extern "C" muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, c
       t.blk_prefix[cnt] = tot;
       return tot;
     };
-    cudaError_t e;
     blocks(0);
-    if ((e = launch_vecop(t, 0, 0, 0, scal, st)) != cudaSuccess) return MUON_ERR_CUDA;   // v = 1/sqrt(cols)
+    if (launch_vecop(t, 0, 0, 0, scal, st) != cudaSuccess) return MUON_ERR_CUDA;   // v = 1/sqrt(cols)
     for (int it = 0; it < cfg->power_iters; ++it) {
       int nb = blocks(1);
-      if ((e = launch_matvec(t, nb, 0, st)) != cudaSuccess) return MUON_ERR_CUDA;     // t = A v
+      if (launch_matvec(t, nb, 0, st) != cudaSuccess) return MUON_ERR_CUDA;     // t = A v
       nb = blocks(2);
-      if ((e = launch_matvec(t, nb, 1, st)) != cudaSuccess) return MUON_ERR_CUDA;     // w = A^T t
+      if (launch_matvec(t, nb, 1, st) != cudaSuccess) return MUON_ERR_CUDA;     // w = A^T t
       blocks(0);
-      if ((e = launch_vecop(t, 0, 1, 0, scal, st)) != cudaSuccess) return MUON_ERR_CUDA;  // v = w / |w|
+      if (launch_vecop(t, 0, 1, 0, scal, st) != cudaSuccess) return MUON_ERR_CUDA;  // v = w / |w|
     }
     int nb = blocks(1);
-    if ((e = launch_matvec(t, nb, 0, st)) != cudaSuccess) return MUON_ERR_CUDA;       // t = A v
+    if (launch_matvec(t, nb, 0, st) != cudaSuccess) return MUON_ERR_CUDA;       // t = A v
     blocks(0);
-    if ((e = launch_vecop(t, 1, 2, 1, scal, st)) != cudaSuccess) return MUON_ERR_CUDA;  // sigma = |t|
-    if (sigma_out && (e = launch_sigma_out(t, scal, sigma_out, st)) != cudaSuccess) return MUON_ERR_CUDA;
+    if (launch_vecop(t, 1, 2, 1, scal, st) != cudaSuccess) return MUON_ERR_CUDA;  // sigma = |t|
+    if (sigma_out && launch_sigma_out(t, scal, sigma_out, st) != cudaSuccess) return MUON_ERR_CUDA;
     if (out) {
-      if ((e = launch_scalars(t, 3, 0, 0.f, 0.f, 0.f, scal, st)) != cudaSuccess) return MUON_ERR_CUDA;
+      if (launch_scalars(t, 3, 0, 0.f, 0.f, 0.f, scal, st) != cudaSuccess) return MUON_ERR_CUDA;
       int tiles = 0;
       for (int k = 0; k < cnt; ++k) {
         MatDesc& d = t.mats[k];
@@ -149,7 +148,7 @@ extern "C" muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, c
         tiles += d.nblk;
       }
       t.blk_prefix[cnt] = tiles;
-      if ((e = launch_epilogue(t, tiles, 0.f, 0, scal, st)) != cudaSuccess) return MUON_ERR_CUDA;
+      if (launch_epilogue(t, tiles, 0.f, 0, scal, st) != cudaSuccess) return MUON_ERR_CUDA;
     }
   }
   return MUON_OK;
