@@ -535,24 +535,63 @@ def main():
     ms_per_step = ms / args.steps
     steps_per_s = 1e3 / ms_per_step
 
-    # ---- end to end: grads host->device from pinned memory, step, params device->host
+    # ---- end to end: grads host->device from pinned memory, step, params device->host.
+    # Every step's grads are copied in and its updated params copied out
+    # inside the timed region, pipelined the way a training loop would run it:
+    # the next step's grads go into a second device buffer on an input copy
+    # stream while this step computes, and the updated params are snapshotted
+    # on the device (one device-to-device copy) and read back on an output
+    # copy stream while the next step runs.  The region ends after the last
+    # read-back has landed in host memory.
     e2e = None
     if not args.no_e2e:
         g_pin = [G_host[k].pin_memory() for k in range(len(owned))]
         p_pin = [torch.empty(shapes[i], dtype=pdt).pin_memory() for i in owned]
         h2d = sum(t.numel() * t.element_size() for t in g_pin)
         d2h = sum(t.numel() * t.element_size() for t in p_pin)
+        gbuf = [grads, [torch.empty_like(g) for g in grads]]
+        snap = [torch.empty_like(q) for q in params]
+        cs_in = torch.cuda.Stream(device=dev)
+        cs_out = torch.cuda.Stream(device=dev)
+        h2d_done = [torch.cuda.Event(), torch.cuda.Event()]
+        used = [torch.cuda.Event(), torch.cuda.Event()]
+        snap_ready, snap_free = torch.cuda.Event(), torch.cuda.Event()
         barrier()
         torch.cuda.synchronize()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
         f0.record(stream)
-        for _ in range(args.steps):
+        cs_in.wait_event(f0)
+
+        def copy_in(b):
+            with torch.cuda.stream(cs_in):
+                for k in range(len(owned)):
+                    gbuf[b][k].copy_(g_pin[k], non_blocking=True)
+                h2d_done[b].record(cs_in)
+
+        copy_in(0)
+        for s_ in range(args.steps):
+            b = s_ % 2
+            if s_ + 1 < args.steps:
+                if s_ >= 1:
+                    cs_in.wait_event(used[1 - b])      # step s_-1 has consumed that buffer
+                copy_in(1 - b)
+            stream.wait_event(h2d_done[b])
+            A.muon_step(cfg, params, gbuf[b], mom, None, ws, stream)
+            if world > 1:
+                SH.exchange(flat, layout, rank)
+            used[b].record(stream)
+            if s_ >= 1:
+                stream.wait_event(snap_free)           # the previous read-back is done with snap
             for k in range(len(owned)):
-                grads[k].copy_(g_pin[k], non_blocking=True)
-            step()
-            for k in range(len(owned)):
-                p_pin[k].copy_(params[k], non_blocking=True)
+                snap[k].copy_(params[k], non_blocking=True)
+            snap_ready.record(stream)
+            cs_out.wait_event(snap_ready)
+            with torch.cuda.stream(cs_out):
+                for k in range(len(owned)):
+                    p_pin[k].copy_(snap[k], non_blocking=True)
+                snap_free.record(cs_out)
+        stream.wait_event(snap_free)
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -562,7 +601,9 @@ def main():
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
         e2e = {"value": 1e3 * args.steps / ems, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h}
+               "d2h_bytes_per_step": d2h,
+               "copies": "every step's grads in and params out, overlapped with compute on two copy streams "
+                         "(double-buffered grads, device snapshot of the params)"}
         if world > 1:
             tot = torch.tensor([h2d, d2h], dtype=torch.float64, device=dev)
             dist.all_reduce(tot)
