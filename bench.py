@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", default="bf16", choices=["bf16", "fp32", "bf16simt"])
+    ap.add_argument("--graph", action="store_true",
+                    help="one GPU: capture the step in a CUDA graph and time its replays (for launch-bound "
+                         "workloads); the per-stage figures then come from one eager step after the timed region")
     ap.add_argument("--ns-vs-cublas", action="store_true",
                     help="time one Newton-Schulz polar of the workload's matrices on this library (ns_polar) "
                          "and the same iteration on torch/cuBLAS bf16 bmm, alternating; prints one JSON line")
@@ -505,6 +508,21 @@ def main():
     torch.cuda.synchronize()
     if A.last_device_status(stream) != A.MUON_OK:
         raise SystemExit("device status error during warm-up")
+    graph = None
+    if args.graph:
+        if world > 1:
+            raise SystemExit("--graph is for one GPU")
+        # the step issues only kernel launches on its stream: capture one and replay it
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            A.muon_step(cfg, params, grads, mom, None, ws)
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        eager_step = step
+
+        def step():
+            graph.replay()
 
     # ---- timed region (device time, CUDA events on the launch stream)
     try:
@@ -528,6 +546,16 @@ def main():
     A.profile_enable(False)
     prof = A.profile_read()
     ms = e0.elapsed_time(e1)
+    if graph is not None:
+        # replays record no per-launch events: take the stage split from one eager step
+        A.profile_enable(True)
+        eager_step()
+        torch.cuda.synchronize()
+        A.profile_enable(False)
+        prof = A.profile_read()
+        for v in prof.values():
+            for k in ("launches", "ms", "flops", "bytes"):
+                v[k] = v[k] * args.steps
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
