@@ -20,9 +20,9 @@
 // both cases, where separate row-dot and column-dot passes take eleven.
 //
 // Kernel k_gramvec: a block owns a range of rows of one matrix (an "item");
-// its thread 0 streams the rows into a ring of shared-memory stages with
-// bulk asynchronous copies (cp.async.bulk, completion on an mbarrier); the
-// 16 warps form teams of TW warps, one row per team per stage, each
+// its thread 0 streams the rows into a 4-stage ring of shared-memory stages
+// with bulk asynchronous copies (cp.async.bulk, completion on an mbarrier);
+// the 16 warps form teams of TW warps, R = 2 rows per team per stage, each
 // thread holding 8-column chunks of y and of the X^T z accumulator in
 // registers.  The row dot is a warp sum, plus an mbarrier-synchronised sum
 // over the team's warps when TW > 1.  Each item writes one partial X^T z
