@@ -8,7 +8,9 @@
 //   [aurora]  D init from the tall-oriented row norms of u
 //   polar loop: scaled input X0 -> rho; ns_steps x {Gram, square, update}
 //               [aurora, not last] D update from the row norms of U
-//   <U,U>, <U,u> -> per-matrix coefficients -> fused epilogue W <- W - lr V
+//   <U,U>, <U,u> (tensor-core mode: formed by the last update GEMM of each
+//   matrix's final polar) -> per-matrix coefficients -> fused epilogue
+//   W <- W - lr V
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
