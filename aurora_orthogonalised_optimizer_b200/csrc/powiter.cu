@@ -250,10 +250,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
     const int64_t row0 = r0 + (int64_t)g * rows_per_group;
     const int nrows = (int)min((int64_t)rows_per_group, r1 - row0);
     const uint32_t fb = s_u32(&ctl->full[s]);
+    // the group's rows are consecutive in X and in the stage: one copy (one
+    // large bulk copy streams faster than one per row, and far faster than
+    // smaller pieces)
     mb_expect_tx(fb, (uint32_t)nrows * row_bytes);
-    for (int k = 0; k < nrows; ++k)
-      bulk_g2s(ring + (uint32_t)s * kGvStageBytes + (uint32_t)k * row_bytes, src + (row0 + k) * (int64_t)row_bytes,
-               row_bytes, fb);
+    bulk_g2s(ring + (uint32_t)s * kGvStageBytes, src + row0 * (int64_t)row_bytes, (uint32_t)nrows * row_bytes, fb);
   };
   int issued = 0;
   if (threadIdx.x == 0)
