@@ -439,9 +439,10 @@ __global__ void __launch_bounds__(512) k_gv_reduce(const MatTable t, int normali
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const float* p = d.gvp + 8 * (int64_t)c;
-    for (int q = 0; q < P; ++q) {
-      const float4 a = reinterpret_cast<const float4*>(p + (int64_t)q * d.ldl)[0];
-      const float4 b = reinterpret_cast<const float4*>(p + (int64_t)q * d.ldl)[1];
+#pragma unroll 6
+    for (int q = 0; q < P; ++q) {   // item order: the sum is the same on every run
+      const float4 a = __ldg(reinterpret_cast<const float4*>(p + (int64_t)q * d.ldl));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(p + (int64_t)q * d.ldl) + 1);
       v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
       v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
     }
