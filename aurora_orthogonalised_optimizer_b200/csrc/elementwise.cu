@@ -493,6 +493,85 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
   }
 }
 
+// Tall matrices whose edges are multiples of 64, bf16 params and bf16
+// Newton-Schulz storage (the common case): the same epilogue with every load
+// issued one tile ahead of its use (packed bf16 in registers), and two shared
+// tiles so each tile needs one barrier.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&v)[8]) {
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    v[2 * h] = __uint_as_float(ww[h] << 16);
+    v[2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads, 3)
+k_epilogue_tall_bf16(const MatTable t, float lr, int update_w, const double* scal) {
+  __shared__ float tV[2][kTile][kTile + 1];
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t tiles_c = d.n / kTile;
+  const int nt = (int)((d.m / kTile) * tiles_c);
+  const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  const int b1 = min(b0 + kEwTilesPerCta, nt);
+  const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
+  const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
+  const bool need_U = cU != 0.f, need_u = cu != 0.f;
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+  const __nv_bfloat16* W = reinterpret_cast<const __nv_bfloat16*>(d.W);
+  const __nv_bfloat16* UX = reinterpret_cast<const __nv_bfloat16*>(d.UX);
+  const __nv_bfloat16* uX = reinterpret_cast<const __nv_bfloat16*>(d.uX);
+  // per tile: W rows r0 + rg (+32) at columns c0 + 8 cg; X rows c0 + rg (+32)
+  // of U and u at columns r0 + 8 cg
+  auto load = [&](int b, uint4 (&w)[2], uint4 (&xU)[2], uint4 (&xu)[2]) {
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t i = r0 + rg + 32 * k, xi = c0 + rg + 32 * k;
+      w[k] = update_w ? __ldg(reinterpret_cast<const uint4*>(W + i * d.n + c0 + 8 * cg)) : make_uint4(0, 0, 0, 0);
+      xU[k] = need_U ? __ldg(reinterpret_cast<const uint4*>(UX + xi * d.ldl + r0 + 8 * cg)) : make_uint4(0, 0, 0, 0);
+      xu[k] = need_u ? __ldg(reinterpret_cast<const uint4*>(uX + xi * d.ldl + r0 + 8 * cg)) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto process = [&](int b, int buf, const uint4 (&w)[2], const uint4 (&xU)[2], const uint4 (&xu)[2]) {
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      float U[8], u[8];
+      bf16x8_to_f32(xU[k], U);
+      bf16x8_to_f32(xu[k], u);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tV[buf][rg + 32 * k][8 * cg + e] = cU * U[e] + cu * u[e];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t ro = (r0 + rg + 32 * k) * d.n + c0 + 8 * cg;
+      float v[8], wf[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = tV[buf][8 * cg + e][rg + 32 * k];
+      if (d.V) st8(d.V, ro, kF32, v);
+      if (update_w) {
+        bf16x8_to_f32(w[k], wf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) wf[e] -= lr * v[e];
+        st8(d.W, ro, kBF16, wf);
+      }
+    }
+  };
+  if (b0 >= b1) return;
+  uint4 wa[2], Ua[2], ua[2], wb[2], Ub[2], ub[2];
+  load(b0, wa, Ua, ua);
+  for (int b = b0; b < b1; b += 2) {
+    if (b + 1 < b1) load(b + 1, wb, Ub, ub);
+    process(b, 0, wa, Ua, ua);
+    if (b + 1 >= b1) break;
+    if (b + 2 < b1) load(b + 2, wa, Ua, ua);
+    process(b + 1, 1, wb, Ub, ub);
+  }
+}
+
 // ============================================================================
 // Flat streaming variants for matrices whose rows are contiguous and a
 // multiple of 8 elements long (no transposition needed): a block walks
@@ -786,6 +865,12 @@ cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w,
                             cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   k_epilogue<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
+  return cudaGetLastError();
+}
+cudaError_t launch_epilogue_tall_bf16(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
+                                      cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_epilogue_tall_bf16<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
   return cudaGetLastError();
 }
 cudaError_t launch_sumsq_wv(const MatTable& t, int nblk, double* partials, cudaStream_t st) {

@@ -681,7 +681,16 @@ muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool updat
     ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_epilogue_flat(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
   }));
-  CK(for_chunks(c, fl.second, blocks_orig, [&](const MatTable& t, int nb) {
+  // tall matrices: the prefetching bf16 kernel when the edges are whole tiles
+  const bool bf16_both = c.param_dtype == kBF16 && c.plan->ns_dtype == kBF16;
+  const auto tl = split_ids(c, fl.second, [bf16_both](const MatDesc& d) {
+    return bf16_both && d.tall && d.m % 64 == 0 && d.n % 64 == 0 && d.ldl == d.m;
+  });
+  CK(for_chunks(c, tl.first, blocks_orig, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
+    return launch_epilogue_tall_bf16(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
+  }));
+  CK(for_chunks(c, tl.second, blocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_epilogue(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
   }));
