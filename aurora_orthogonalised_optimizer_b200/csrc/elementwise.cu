@@ -658,6 +658,64 @@ k_scale_cols_flat(const MatTable t, double* partials) {
   }
 }
 
+// bf16 Newton-Schulz storage: the same scaling with each chunk's loads (u
+// and the column scales) issued while the previous chunk is processed.
+__global__ void __launch_bounds__(kEwThreads)
+k_scale_cols_flat_bf16(const MatTable t, double* partials) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t total = d.s * d.l;
+  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  const int64_t c1 = min(c0 + kEwTilesPerCta, (total + kFlatChunk - 1) / kFlatChunk);
+  const __nv_bfloat16* uX = reinterpret_cast<const __nv_bfloat16*>(d.uX);
+  auto off = [&](int64_t c, int k) { return c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k); };
+  auto load = [&](int64_t c, uint4 (&x)[2], float4 (&dj)[2][2]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = off(c, k);
+      if (e < total) {
+        x[k] = __ldg(reinterpret_cast<const uint4*>(uX + e));
+        const float4* dp = reinterpret_cast<const float4*>(d.D + e % d.l);
+        dj[k][0] = __ldg(dp);
+        dj[k][1] = __ldg(dp + 1);
+      } else {
+        x[k] = make_uint4(0, 0, 0, 0);
+        dj[k][0] = dj[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
+  auto process = [&](int64_t c, const uint4 (&x)[2], const float4 (&dj)[2][2]) {
+    float s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = off(c, k);
+      if (e >= total) continue;
+      float v[8];
+      bf16x8_to_f32(x[k], v);
+      const float dd[8] = {dj[k][0].x, dj[k][0].y, dj[k][0].z, dj[k][0].w,
+                           dj[k][1].x, dj[k][1].y, dj[k][1].z, dj[k][1].w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[q] *= dd[q];
+        s2 += v[q] * v[q];
+      }
+      st8(d.X0, e, kBF16, v);
+    }
+    warp_partials(partials, d.part + c, 1, s2, 0.f);
+  };
+  if (c0 >= c1) return;
+  uint4 xa[2], xb[2];
+  float4 da[2][2], db[2][2];
+  load(c0, xa, da);
+  for (int64_t c = c0; c < c1; c += 2) {
+    if (c + 1 < c1) load(c + 1, xb, db);
+    process(c, xa, da);
+    if (c + 1 >= c1) break;
+    if (c + 2 < c1) load(c + 2, xa, da);
+    process(c + 1, xb, db);
+  }
+}
+
 __global__ void __launch_bounds__(kEwThreads)
 k_dots_flat(const MatTable t, double* partials) {
   const int mi = find_mat(t, blockIdx.x);
@@ -724,6 +782,64 @@ k_epilogue_flat(const MatTable t, float lr, int update_w, const double* scal) {
       if (d.V) st8(d.V, e, kF32, v);
       if (update_w) st8(d.W, e, t.param_dtype, w[k]);
     }
+  }
+}
+
+// bf16 params and bf16 Newton-Schulz storage: the same flat epilogue with
+// each chunk's loads issued while the previous chunk is processed.
+__global__ void __launch_bounds__(kEwThreads)
+k_epilogue_flat_bf16(const MatTable t, float lr, int update_w, const double* scal) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t total = d.m * d.n;
+  const float cU = (float)scal[d.idx * S_COUNT + S_COEF_U];
+  const float cu = (float)scal[d.idx * S_COUNT + S_COEF_u];
+  const bool need_U = cU != 0.f, need_u = cu != 0.f;
+  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  const int64_t c1 = min(c0 + kEwTilesPerCta, (total + kFlatChunk - 1) / kFlatChunk);
+  const __nv_bfloat16* UX = reinterpret_cast<const __nv_bfloat16*>(d.UX);
+  const __nv_bfloat16* uX = reinterpret_cast<const __nv_bfloat16*>(d.uX);
+  const __nv_bfloat16* W = reinterpret_cast<const __nv_bfloat16*>(d.W);
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  // element offset of group k of chunk c for this thread (total is a multiple of 8)
+  auto off = [&](int64_t c, int k) { return c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k); };
+  auto load = [&](int64_t c, uint4 (&a)[2], uint4 (&b)[2], uint4 (&w)[2]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = off(c, k);
+      const bool in = e < total;
+      a[k] = in && need_U ? __ldg(reinterpret_cast<const uint4*>(UX + e)) : z4;
+      b[k] = in && need_u ? __ldg(reinterpret_cast<const uint4*>(uX + e)) : z4;
+      w[k] = in && update_w ? __ldg(reinterpret_cast<const uint4*>(W + e)) : z4;
+    }
+  };
+  auto process = [&](int64_t c, const uint4 (&a)[2], const uint4 (&b)[2], const uint4 (&w)[2]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = off(c, k);
+      if (e >= total) continue;
+      float U[8], u[8], wf[8], v[8];
+      bf16x8_to_f32(a[k], U);
+      bf16x8_to_f32(b[k], u);
+      bf16x8_to_f32(w[k], wf);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[q] = cU * U[q] + cu * u[q];
+        wf[q] -= lr * v[q];
+      }
+      if (d.V) st8(d.V, e, kF32, v);
+      if (update_w) st8(d.W, e, kBF16, wf);
+    }
+  };
+  if (c0 >= c1) return;
+  uint4 aa[2], ba[2], wa[2], ab[2], bb[2], wb[2];
+  load(c0, aa, ba, wa);
+  for (int64_t c = c0; c < c1; c += 2) {
+    if (c + 1 < c1) load(c + 1, ab, bb, wb);
+    process(c, aa, ba, wa);
+    if (c + 1 >= c1) break;
+    if (c + 2 < c1) load(c + 2, aa, ba, wa);
+    process(c + 1, ab, bb, wb);
   }
 }
 
@@ -865,6 +981,17 @@ cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w,
                             cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   k_epilogue<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
+  return cudaGetLastError();
+}
+cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_scale_cols_flat_bf16<<<nblk, kEwThreads, 0, st>>>(t, partials);
+  return cudaGetLastError();
+}
+cudaError_t launch_epilogue_flat_bf16(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
+                                      cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_epilogue_flat_bf16<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
   return cudaGetLastError();
 }
 cudaError_t launch_epilogue_tall_bf16(const MatTable& t, int nblk, float lr, int update_w, const double* scal,

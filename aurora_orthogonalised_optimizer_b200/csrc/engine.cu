@@ -635,7 +635,8 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       const auto fx = split_ids(c, eq_ids, flat_x);
       CK(for_chunks(c, fx.first, fblocks_x, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
-        return launch_scale_cols_flat(t, nb, c.partials, c.st);
+        return c.plan->ns_dtype == kBF16 ? launch_scale_cols_flat_bf16(t, nb, c.partials, c.st)
+                                         : launch_scale_cols_flat(t, nb, c.partials, c.st);
       }));
       CK(for_chunks(c, fx.second, blocks_x, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
@@ -677,12 +678,14 @@ muon_status stage_epilogue(const Ctx& c, const std::vector<int>& ids, bool updat
   const double per_elem = c.plan->nsb * (need_u ? 2.0 : 1.0) + (update_w ? 2.0 * dt_bytes(c.param_dtype) : 0.0) +
                           (c.V ? 4.0 : 0.0);
   const auto fl = split_ids(c, ids, flat_orig);
+  // bf16 params and NS storage: the kernels that load one chunk / tile ahead
+  const bool bf16_both = c.param_dtype == kBF16 && c.plan->ns_dtype == kBF16;
   CK(for_chunks(c, fl.first, fblocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_EPILOGUE, 0.0, per_elem * table_elems(t), c.st);
-    return launch_epilogue_flat(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
+    return bf16_both ? launch_epilogue_flat_bf16(t, nb, lr, update_w ? 1 : 0, c.scal, c.st)
+                     : launch_epilogue_flat(t, nb, lr, update_w ? 1 : 0, c.scal, c.st);
   }));
   // tall matrices: the prefetching bf16 kernel when the edges are whole tiles
-  const bool bf16_both = c.param_dtype == kBF16 && c.plan->ns_dtype == kBF16;
   const auto tl = split_ids(c, fl.second, [bf16_both](const MatDesc& d) {
     return bf16_both && d.tall && d.m % 64 == 0 && d.n % 64 == 0 && d.ldl == d.m;
   });
