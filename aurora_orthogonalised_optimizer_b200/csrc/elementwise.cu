@@ -785,6 +785,85 @@ k_epilogue_flat(const MatTable t, float lr, int update_w, const double* scal) {
   }
 }
 
+// Optimizer-step prologue for tall matrices whose edges are multiples of 64,
+// bf16 grads, params and Newton-Schulz storage: the same arithmetic as
+// k_prologue with each tile's loads issued while the previous tile is
+// processed, and two shared tiles (one barrier per tile).
+__global__ void __launch_bounds__(kEwThreads, 2)
+k_prologue_tall_bf16(const MatTable t, float mu, int nesterov, int want_w2, double* partials) {
+  __shared__ float tile[2][kTile][kTile + 1];
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t tiles_c = d.n / kTile;
+  const int nt = (int)((d.m / kTile) * tiles_c);
+  const int b0 = (blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  const int b1 = min(b0 + kEwTilesPerCta, nt);
+  const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+  const __nv_bfloat16* G = reinterpret_cast<const __nv_bfloat16*>(d.G);
+  const __nv_bfloat16* W = reinterpret_cast<const __nv_bfloat16*>(d.W);
+  struct Raw { uint4 g[2]; float4 m[2][2]; uint4 w[2]; };
+  auto load = [&](int b, Raw& r) {
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = (r0 + rg + 32 * k) * d.n + c0 + 8 * cg;
+      r.g[k] = __ldg(reinterpret_cast<const uint4*>(G + e));
+      r.m[k][0] = reinterpret_cast<const float4*>(d.M + e)[0];
+      r.m[k][1] = reinterpret_cast<const float4*>(d.M + e)[1];
+      r.w[k] = want_w2 ? __ldg(reinterpret_cast<const uint4*>(W + e)) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto process = [&](int b, int buf, const Raw& r) {
+    const int64_t r0 = (b / tiles_c) * kTile, c0 = (b % tiles_c) * kTile;
+    float g[2][8], m[2][8], w[2][8], u[2][8];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      bf16x8_to_f32(r.g[k], g[k]);
+      bf16x8_to_f32(r.w[k], w[k]);
+      m[k][0] = r.m[k][0].x; m[k][1] = r.m[k][0].y; m[k][2] = r.m[k][0].z; m[k][3] = r.m[k][0].w;
+      m[k][4] = r.m[k][1].x; m[k][5] = r.m[k][1].y; m[k][6] = r.m[k][1].z; m[k][7] = r.m[k][1].w;
+    }
+    float su2 = 0.f, sw2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        m[k][e] = m[k][e] + (1.f - mu) * (g[k][e] - m[k][e]);
+        u[k][e] = nesterov ? g[k][e] + mu * (m[k][e] - g[k][e]) : m[k][e];
+      }
+      su2 += u[0][e] * u[0][e] + u[1][e] * u[1][e];
+      sw2 += w[0][e] * w[0][e] + w[1][e] * w[1][e];
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      st8(d.M, (r0 + rg + 32 * k) * d.n + c0 + 8 * cg, kF32, m[k]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tile[buf][rg + 32 * k][8 * cg + e] = u[k][e];
+    }
+    __syncthreads();
+    // X row = original column c0 + xr; X columns = original rows r0 + 8 cg ..
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int xr = rg + 32 * k;
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = tile[buf][8 * cg + e][xr];
+      st8(d.uX, (c0 + xr) * d.ldl + r0 + 8 * cg, kBF16, v);
+    }
+    warp_partials(partials, d.part + b, 2, su2, sw2);
+  };
+  if (b0 >= b1) return;
+  Raw ra, rb;
+  load(b0, ra);
+  for (int b = b0; b < b1; b += 2) {
+    if (b + 1 < b1) load(b + 1, rb);
+    process(b, 0, ra);
+    if (b + 1 >= b1) break;
+    if (b + 2 < b1) load(b + 2, ra);
+    process(b + 1, 1, rb);
+  }
+}
+
 // bf16 params and bf16 Newton-Schulz storage: the same flat epilogue with
 // each chunk's loads issued while the previous chunk is processed.
 __global__ void __launch_bounds__(kEwThreads)
@@ -981,6 +1060,12 @@ cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w,
                             cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   k_epilogue<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
+  return cudaGetLastError();
+}
+cudaError_t launch_prologue_tall_bf16(const MatTable& t, int nblk, float mu, int nesterov, int want_w2,
+                                      double* partials, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_prologue_tall_bf16<<<nblk, kEwThreads, 0, st>>>(t, mu, nesterov, want_w2, partials);
   return cudaGetLastError();
 }
 cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st) {

@@ -378,7 +378,17 @@ muon_status stage_prologue(const Ctx& c, const std::vector<int>& ids, int mode, 
     ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_prologue_flat(t, nb, mode, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
   }));
-  CK(for_chunks(c, fl.second, blocks_orig, [&](const MatTable& t, int nb) {
+  // tall: the bf16 kernel that loads one tile ahead when the edges are whole tiles
+  const bool bf16_all = mode == 0 && c.grad_dtype == kBF16 && c.plan->ns_dtype == kBF16 &&
+                        (!want_w2 || c.param_dtype == kBF16);
+  const auto tl = split_ids(c, fl.second, [bf16_all](const MatDesc& d) {
+    return bf16_all && d.tall && d.m % 64 == 0 && d.n % 64 == 0 && d.ldl == d.m;
+  });
+  CK(for_chunks(c, tl.first, blocks_orig, [&](const MatTable& t, int nb) {
+    ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
+    return launch_prologue_tall_bf16(t, nb, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
+  }));
+  CK(for_chunks(c, tl.second, blocks_orig, [&](const MatTable& t, int nb) {
     ProfScope ps(PC_PROLOGUE, 0.0, per_elem * table_elems(t), c.st);
     return launch_prologue(t, nb, mode, c.cfg->mu, c.cfg->nesterov, want_w2 ? 1 : 0, c.partials, c.st);
   }));

@@ -91,6 +91,9 @@ cudaError_t launch_vecop(const MatTable& t, int which, int mode, int len_is_s_wh
 cudaError_t launch_dots(const MatTable& t, int nblk, double* partials, cudaStream_t st);
 cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
                             cudaStream_t st);
+// Optimizer-step prologue, tall, m and n multiples of 64, bf16 grads / params / NS storage.
+cudaError_t launch_prologue_tall_bf16(const MatTable& t, int nblk, float mu, int nesterov, int want_w2,
+                                      double* partials, cudaStream_t st);
 // Flat Aurora input scaling with bf16 NS storage.
 cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st);
 // Flat (wide / square, rows a multiple of 8) and bf16 params and NS storage.
