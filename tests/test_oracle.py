@@ -309,6 +309,22 @@ def test_floor_triggers_on_heavy_weights():
     assert np.linalg.norm(V) / np.linalg.norm(W) == pytest.approx(wl.cfg.target_uw, rel=1e-12)
 
 
+@pytest.mark.parametrize("shape", [(256, 128), (96, 160), (64, 64)])
+def test_zero_gradient_step_leaves_weights_unchanged(shape):
+    """Degenerate input: g = 0 from zero momentum.  Every guard (the NS eps,
+    the power-iteration and operator-norm floors, Aurora's pp_eps, the
+    restore's 1e-10, the floor's 1e-8) must keep the step finite, so V = 0
+    and W is returned as it was (a dropped or misplaced eps gives NaN)."""
+    wl = WL.single_aurora_256x128()
+    rng = np.random.default_rng(5)
+    W = rng.standard_normal(shape) * 0.02
+    g = np.zeros(shape)
+    W_new, m_new, V = O.step(W, g, np.zeros(shape), wl.cfg, "f32")
+    assert np.all(np.isfinite(V)) and np.all(V == 0.0)
+    assert np.all(m_new == 0.0)
+    assert np.array_equal(W_new, W.astype(np.float32).astype(np.float64))
+
+
 def test_weight_decay_rejected():
     cfg = WL.aurora_stack(weight_decay=0.1)
     with pytest.raises(ValueError):
