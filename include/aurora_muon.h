@@ -41,7 +41,7 @@ extern "C" {
 typedef enum {
   MUON_OK = 0,
   MUON_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad shape, bad config value */
-  MUON_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement */
+  MUON_ERR_UNSUPPORTED = 2,  /* a valid request the library does not implement */
   MUON_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than muon_workspace_size() */
   MUON_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
   MUON_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up (see muon_last_device_status) */
