@@ -81,10 +81,13 @@ def _worker(rank, world, port, shapes, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_exchange_gives_every_rank_every_update(world):
+@pytest.mark.parametrize("world,shapes", [
+    (2, [(48, 16), (16, 48), (32, 32), (8, 100), (100, 8)]),
+    (3, [(48, 16), (16, 48), (32, 32), (8, 100), (100, 8)]),
+    (3, [(48, 16), (16, 48)]),                          # one rank owns nothing
+])
+def test_exchange_gives_every_rank_every_update(world, shapes):
     import torch.multiprocessing as mp
-    shapes = [(48, 16), (16, 48), (32, 32), (8, 100), (100, 8)]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
