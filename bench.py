@@ -162,7 +162,7 @@ def oracle_sample_time(wl, indices):
 
 def sample_indices(wl):
     if wl.name.startswith("llama"):
-        return [0, 1, 2]                       # layer 0: q (3072^2), k, v (1024 x 3072)
+        return [0, 1, 2, 3, 6, 7, 8, 9]        # layers 0 and 1: q, o (3072^2), k, v (1024 x 3072)
     if wl.n <= 8:
         return list(range(wl.n))
     return [0, 1]
