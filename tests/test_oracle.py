@@ -309,6 +309,95 @@ def test_floor_triggers_on_heavy_weights():
     assert np.linalg.norm(V) / np.linalg.norm(W) == pytest.approx(wl.cfg.target_uw, rel=1e-12)
 
 
+def _hadamard(n):
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def _grad_for_blend(u_star, m0, mu):
+    """The gradient whose Nesterov blend with momentum m0 is exactly u_star.
+
+    With m' = m0 + (1 - mu)(g - m0) and u = g + mu (m' - g), u is
+    (1 - mu^2) g + mu^2 m0, so g = (u_star - mu^2 m0) / (1 - mu^2)."""
+    return (u_star - mu * mu * m0) / (1.0 - mu * mu)
+
+
+def _power_closed_form(s, Qr, n, iters):
+    """sigma-hat of the power iteration from v0 = ones(n)/sqrt(n), by its spectral form."""
+    c = Qr.T @ np.full(n, 1.0 / math.sqrt(n))
+    wts = s ** (2 * iters) * c
+    return np.linalg.norm(s * wts) / np.linalg.norm(wts)
+
+
+def _contra_closed_form(s, sigma, contra):
+    """Singular values of restore(U - contra/2 * u/sigma) when U = Q P^T and u = Q diag(s) P^T."""
+    d = 1.0 - 0.5 * contra * s / sigma
+    return d * math.sqrt(len(s)) / np.linalg.norm(d)
+
+
+def test_step_composition_with_momentum_plain_ns_closed_form():
+    """Composition of the update ([T3] 组合优化栈 / Contra-Muon) with non-zero
+    momentum, so that the Nesterov blend u is not a multiple of g.
+
+    g is chosen so the blend is exactly u* = Q diag(s) P^T (condition 8).  The
+    converged polar of u* is Q P^T, sigma-hat has its spectral closed form, so
+    V = Q diag(d) P^T * aspect with d from the restore of 1 - (C/2) s / sigma.
+    Fails if N is taken from U or from g, if g (not u) goes into the polar, or
+    if the aspect factor is applied before the restore."""
+    rng = np.random.default_rng(40)
+    m, n = 24, 10
+    s = np.linspace(1.0, 8.0, n)[rng.permutation(n)]
+    u_star, Ql, Qr = _with_spectrum(rng, m, n, s)
+    m0 = rng.standard_normal((m, n))
+    cfg = WL.plain_muon(contra=0.4, power_iters=5, mu=0.9, ns_steps=12)
+    g = _grad_for_blend(u_star, m0, cfg.mu)
+    V, m_new, parts = O.muon_update(g, m0, cfg, return_parts=True)
+    assert np.allclose(parts["u"], u_star, atol=1e-12)
+    assert np.allclose(m_new, m0 + (1.0 - cfg.mu) * (g - m0), atol=1e-12)
+    sigma = _power_closed_form(s, Qr, n, cfg.power_iters)
+    assert parts["sigma"] == pytest.approx(sigma, rel=1e-10)
+    want = math.sqrt(m / n) * Ql @ np.diag(_contra_closed_form(s, sigma, cfg.contra)) @ Qr.T
+    assert np.allclose(V, want, atol=1e-8)
+    # the blend is far from a multiple of g, so the slips above are visible
+    cosine = np.sum(g * u_star) / (np.linalg.norm(g) * np.linalg.norm(u_star))
+    assert cosine < 0.9
+
+
+def test_step_composition_with_momentum_aurora_wide_closed_form():
+    """The same composition with Aurora on a wide matrix.
+
+    u* = Q diag(s) P^T with P = columns of a Hadamard matrix / sqrt(n): every
+    column of u* has the same norm and every row of P has norm^2 m/n (the
+    Aurora target), so D stays constant and Aurora(u*) = Q P^T ([T3] 要点解释:
+    row norms already equal are a fixed point).  The all-ones column of H is
+    one of P's columns, so the power iteration from ones/sqrt(n) sees only
+    its singular value: sigma-hat = s[j0] exactly (not sigma_max).  Aurora of
+    g instead of u*, N from U, or N from g all change V."""
+    rng = np.random.default_rng(41)
+    m, n = 6, 16
+    H = _hadamard(n)
+    cols = [3, 0, 9, 5, 12, 6]                 # H's all-ones column sits at position 1
+    P = H[:, cols] / math.sqrt(n)
+    Q = _orth(rng, m, m)
+    s = np.array([2.0, 3.0, 5.0, 1.5, 4.0, 2.5])
+    u_star = Q @ np.diag(s) @ P.T
+    m0 = rng.standard_normal((m, n))
+    cfg = WL.aurora_stack(mu=0.95, target_uw=0.0)
+    g = _grad_for_blend(u_star, m0, cfg.mu)
+    # the construction: equal column norms of u*, and Aurora(u*) is the plain polar
+    assert np.allclose(np.linalg.norm(u_star, axis=0), np.linalg.norm(s) / math.sqrt(n), rtol=1e-12)
+    V, _, parts = O.muon_update(g, m0, cfg, return_parts=True)
+    assert np.allclose(parts["u"], u_star, atol=1e-12)
+    assert parts["sigma"] == pytest.approx(s[1], rel=1e-12)
+    assert np.allclose(parts["U"], Q @ P.T, atol=1e-8)
+    want = Q @ np.diag(_contra_closed_form(s, s[1], cfg.contra)) @ P.T     # wide: aspect 1
+    assert np.allclose(V, want, atol=1e-8)
+    # Aurora of the raw gradient is a different matrix
+    assert np.linalg.norm(O.aurora_orthogonalize(g) - Q @ P.T) > 0.1
+
+
 @pytest.mark.parametrize("shape", [(256, 128), (96, 160), (64, 64)])
 def test_zero_gradient_step_leaves_weights_unchanged(shape):
     """Degenerate input: g = 0 from zero momentum.  Every guard (the NS eps,
