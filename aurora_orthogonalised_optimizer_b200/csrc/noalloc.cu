@@ -29,7 +29,9 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_opnorm_scratch[kScratchBytes];
 
 // Device address of g_opnorm_scratch on the current device, looked up once
-// per device (with that device current) on the first call made on it.
+// per device (with that device current) on the first call made on it and
+// kept for the life of the process.  A cudaDeviceReset reloads the module
+// and can move the array, so none may come between calls.
 cudaError_t scratch_address(void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
@@ -70,6 +72,9 @@ extern "C" muon_status opnorm_normalize_noalloc(const muon_config* cfg, int n, c
   for (int i = 0; i < n; ++i) {
     const int64_t m = shapes[i].rows, k = shapes[i].cols;
     if (m <= 0 || k <= 0) return MUON_ERR_INVALID_ARG;
+    // the same edge bound as the workspace entry points; it also keeps each
+    // term of the sum below far from wrapping around
+    if (m > (int64_t)1 << 31 || k > (int64_t)1 << 31) return MUON_ERR_INVALID_ARG;
     if (!in[i] || ((uintptr_t)in[i] & 15u)) return MUON_ERR_INVALID_ARG;
     if (out && out[i] && ((uintptr_t)out[i] & 15u)) return MUON_ERR_INVALID_ARG;
     need += sizeof(float) * (round64(k) + round64(m));

@@ -156,7 +156,10 @@ muon_status opnorm_normalize(const muon_config* cfg, int n, const muon_shape* sh
  *    anything is launched.
  *  - Calls no cudaMalloc / cudaFree.  The first call on a device looks up
  *    the array's device address (cudaGetSymbolAddress, with that device
- *    current); make that first call before any stream capture.
+ *    current); make that first call before any stream capture.  The address
+ *    is kept for the life of the process: no cudaDeviceReset may come
+ *    between calls (a reset reloads the module and can move the array).
+ *  - rows or cols above 2^31 return MUON_ERR_INVALID_ARG.
  *  - Every call shares the one array and it keeps the last call's contents;
  *    each call clears its scalar block first.  Calls that overlap on the
  *    GPU (different streams, or different host threads on one device) race

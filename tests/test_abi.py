@@ -164,3 +164,17 @@ def test_size_limits_are_rejected_on_the_host(lib):
     assert _call_step(lib, _cfg(), [(40000, 40000)], p, g, m) == A.MUON_ERR_UNSUPPORTED
     assert A.workspace_size(A.Config(), [(40000, 40000)]) == 0
     assert _call_step(lib, _cfg(), [(1 << 32, 8)], p, g, m) == A.MUON_ERR_INVALID_ARG
+
+
+def test_noalloc_entry_rejects_oversized_edges_on_the_host(lib):
+    """rows or cols above 2^31 are refused before the scratch size is summed
+    (near 2^62 the sum would wrap around and pass the 1 MiB check)."""
+    cfg = A.Config()
+    ptrs = (C.c_void_p * 1)(FAKE)
+    for shape in [((1 << 62) - 64, 8), (8, (1 << 62) - 64), ((1 << 31) + 1, 1)]:
+        code = lib.opnorm_normalize_noalloc(C.byref(cfg.to_c()), 1, A._shapes([shape]), ptrs, A.MUON_F32,
+                                            None, None, None)
+        assert code == A.MUON_ERR_INVALID_ARG, shape
+    code = lib.opnorm_normalize_noalloc(C.byref(cfg.to_c()), 1, A._shapes([(1 << 31, 1 << 31)]), ptrs,
+                                        A.MUON_F32, None, None, None)
+    assert code == A.MUON_ERR_UNSUPPORTED          # inside the edge bound, beyond the scratch

@@ -5,7 +5,8 @@ after start-up).  Its scratch is a static array inside the library, so it
 takes no workspace.  Its output must match the workspace entry point
 opnorm_normalize within the tolerance the other operator-norm tests use, on
 two calls in a row (the second call reuses the static array the first call
-left behind).  This file is collected last on purpose."""
+left behind), and the float64 oracle run on the same stored input values.
+This file is collected last on purpose."""
 import ctypes as C
 
 import numpy as np
@@ -15,9 +16,11 @@ torch = pytest.importorskip("torch")
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
+import oracle.muon_oracle as O  # noqa: E402
 from aurora_orthogonalised_optimizer_b200 import _abi as A  # noqa: E402
 
 TOL = 1e-5          # fp32 inputs, as in the operator-norm parity test
+ORACLE_TOL = 1e-5   # fp32 arithmetic on the stored values against float64
 
 
 def _inputs(shapes, seed, dtype):
@@ -48,6 +51,14 @@ def _compare(cfg, ins):
     for a, b in zip(no, ro):
         rel = (a.double() - b.double()).norm() / b.double().norm()
         assert rel.item() <= TOL, rel.item()
+    # directly against the oracle: the power iteration runs in fp32 on the
+    # stored values, so both dtypes meet the fp32 bound
+    for k, t in enumerate(ins):
+        x = t.double().cpu().numpy()
+        N, s = O.scale_to_unit_operator_norm(x, cfg.power_iters)
+        assert abs(ns[k].item() - s) <= ORACLE_TOL * s, (t.shape, ns[k].item(), s)
+        got = no[k].double().cpu().numpy()
+        assert np.linalg.norm(got - N) <= ORACLE_TOL * np.linalg.norm(N), t.shape
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
