@@ -1,13 +1,18 @@
-"""Full-size parity of the 3.8B matrix set (168 matrices, 2.82 G parameters)
+"""Full-size parity of the 3.8B matrix sets (168 matrices, 2.82 G parameters)
 in the launch configuration the bench times: one muon_step call over every
-matrix, tensor-core Newton-Schulz.
+matrix per step, tensor-core Newton-Schulz, for all 3 steps each set states.
 
-* Sampled outputs: the k and v matrices (1024 x 3072) of the first and the
-  last layer, and (second Aurora test) one fc (12288 x 3072), one proj
-  (3072 x 12288) and one q (3072 x 3072), are recomputed by the float64
-  oracle; update V within 3e-2 relative Frobenius error, momentum within 1e-6.
-* Properties that hold for every matrix at any size, checked on all 168:
-  - first step from zero momentum: m = (1 - mu) g up to fp32 rounding;
+* Sampled outputs: one fc (12288 x 3072, tall), one proj (3072 x 12288,
+  wide), one q (3072 x 3072, square) and k / v (1024 x 3072) of the first
+  and last layer follow the float64 oracle's own trajectory (its weights and
+  momentum carried from step to step); at every step the update V is within
+  3e-2 relative Frobenius error and the momentum within 1e-6.  From step 2 on
+  the momentum is non-zero, so the Nesterov blend u is not a multiple of the
+  gradient and the operands of the polar and of the contra term are told
+  apart.
+* Properties that hold for every matrix at any size, checked on all 168 at
+  every step:
+  - momentum: m = m_prev + (1 - mu)(g - m_prev) up to fp32 rounding;
   - the parameter add: W_new = W - lr V up to the bf16 rounding of W_new
     and the fp32 rounding of the product and the difference;
   - the update is finite and (Aurora stack) ||V||_F / ||W||_F >= TARGET_UW.
@@ -26,27 +31,15 @@ pytestmark = [pytest.mark.gpu,
 from aurora_orthogonalised_optimizer_b200 import _abi as A  # noqa: E402
 
 
-def _run(wl, sample):
-    W, G = WL.generate_torch(wl, None, 0, threads=16)
-    cfg = A.Config.from_step_config(wl.cfg, gemm_mode=A.MUON_GEMM_BF16, param_dtype=A.MUON_BF16,
-                                    grad_dtype=A.MUON_BF16)
-    p = [w.cuda() for w in W]
-    g = [x.cuda() for x in G]
-    m = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
-    v = [torch.empty(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
-    w_before = [t.clone() for t in p]
-    ws = A.make_workspace(cfg, wl.shapes)
-    A.muon_step(cfg, p, g, m, v, ws)
-    torch.cuda.synchronize()
-    assert A.last_device_status() == A.MUON_OK
-    del ws
+def _check_all(wl, p, w_prev, g, m, m_prev, v):
+    """Properties every matrix meets after one step, whatever its size."""
     mu, lr = wl.cfg.mu, wl.cfg.lr
     for k in range(wl.n):
-        gk = g[k].float()
-        assert torch.isfinite(v[k]).all()
-        em = ((m[k] - (1.0 - mu) * gk).norm() / ((1.0 - mu) * gk).norm()).item()
+        assert torch.isfinite(v[k]).all(), ("V not finite", k)
+        want_m = m_prev[k].double() + (1.0 - mu) * (g[k].double() - m_prev[k].double())
+        em = ((m[k].double() - want_m).norm() / want_m.norm()).item()
         assert em <= 1e-6, ("momentum", k, em)
-        w0 = w_before[k].double()
+        w0 = w_prev[k].double()
         step = lr * v[k].double()
         want = w0 - step
         # bf16 rounding of W_new plus the fp32 rounding of lr * V and of the subtraction
@@ -56,33 +49,52 @@ def _run(wl, sample):
         assert bool((err <= bound).all()), ("param add", k, (err / bound).max().item())
         if wl.cfg.target_uw > 0:
             assert (v[k].norm() / w0.norm()).item() >= wl.cfg.target_uw * (1 - 1e-5)
-    # sampled matrices against the oracle
-    for k in sample:
-        Wn, Gn, Mn = WL.generate(wl, [k])
-        _, m_or, V_or = O.step(WL.to_f64(Wn[0], WL.BF16), WL.to_f64(Gn[0], WL.BF16), Mn[0].astype(np.float64),
-                               wl.cfg, WL.BF16)
-        ev = rel_fro(f64(v[k]), V_or)
-        assert ev <= 3e-2, ("V", k, wl.shapes[k], ev)
-        assert rel_fro(f64(m[k]), m_or) <= 1e-6
 
 
-def test_llama_3p8b_aurora_stack_full_size():
-    wl = WL.llama_3p8b_aurora()
-    # k, v of layer 0 and of layer 27 (1024 x 3072, the Aurora wide path)
-    _run(wl, [1, 2, 6 * 27 + 1, 6 * 27 + 2])
+def _run_full(wl, sample):
+    cfg = A.Config.from_step_config(wl.cfg, gemm_mode=A.MUON_GEMM_BF16, param_dtype=A.MUON_BF16,
+                                    grad_dtype=A.MUON_BF16)
+    W, _ = WL.generate_torch(wl, None, 0, threads=16, want_g=False)
+    p = [w.cuda() for w in W]
+    del W
+    m = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    v = [torch.empty(s, dtype=torch.float32, device="cuda") for s in wl.shapes]
+    ws = A.make_workspace(cfg, wl.shapes)
+    Wn, _, _ = WL.generate(wl, sample)
+    oW = {k: WL.to_f64(Wn[j], WL.BF16) for j, k in enumerate(sample)}
+    oM = {k: np.zeros(wl.shapes[k]) for k in sample}
+    assert wl.steps == 3
+    for st in range(wl.steps):
+        _, G = WL.generate_torch(wl, None, st, threads=16, want_w=False)
+        g = [x.cuda() for x in G]
+        del G
+        w_prev = [t.clone() for t in p]
+        m_prev = [t.clone() for t in m]
+        A.muon_step(cfg, p, g, m, v, ws)
+        torch.cuda.synchronize()
+        assert A.last_device_status() == A.MUON_OK
+        _check_all(wl, p, w_prev, g, m, m_prev, v)
+        del w_prev, m_prev, g
+        for k in sample:
+            gk = WL.to_f64(WL.grad(wl, k, st), WL.BF16)
+            oW[k], oM[k], V = O.step(oW[k], gk, oM[k], wl.cfg, WL.BF16)
+            ev = rel_fro(f64(v[k]), V)
+            assert ev <= 3e-2, ("V", st, k, wl.shapes[k], ev)
+            assert rel_fro(f64(m[k]), oM[k]) <= 1e-6, ("m", st, k)
 
 
-def test_llama_3p8b_aurora_stack_full_size_tall_wide_square():
-    wl = WL.llama_3p8b_aurora()
-    # fc of layer 0 (12288 x 3072: tall, transposed into the X orientation,
-    # two Aurora polars), proj of layer 13 (3072 x 12288: wide, two polars)
-    # and q of layer 27 (3072 x 3072: square, one polar)
-    _run(wl, [4, 6 * 13 + 5, 6 * 27])
+# fc of layer 0 (tall: transposed into the X orientation; two Aurora polars),
+# proj of layer 13 (wide, two polars), q of layer 27 (square, one polar),
+# k of layer 0 and v of layer 27 (1024 x 3072, the Aurora wide path)
+SAMPLE = [1, 4, 6 * 13 + 5, 6 * 27, 6 * 27 + 2]
 
 
-def test_llama_3p8b_plain_muon_full_size():
-    wl = WL.llama_3p8b_plain()
-    _run(wl, [1, 6 * 27 + 2])
+def test_llama_3p8b_aurora_stack_full_size_three_steps():
+    _run_full(WL.llama_3p8b_aurora(), SAMPLE)
+
+
+def test_llama_3p8b_plain_muon_full_size_three_steps():
+    _run_full(WL.llama_3p8b_plain(), SAMPLE)
 
 
 def _run_sampled_trajectory(wl, sample, gemm_mode=A.MUON_GEMM_BF16, tol=3e-2):
