@@ -16,15 +16,24 @@ from typing import List, Optional, Sequence
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libaurora_muon.so")
+# AURORA_MUON_CHECKED=1 loads the bounds-checked build of the same library
+# (every kernel's global accesses tested against their buffers' extents).
+CHECKED_LIB_PATH = os.path.join(HERE, "libaurora_muon_checked.so")
 
-MUON_OK, MUON_ERR_INVALID_ARG, MUON_ERR_UNSUPPORTED, MUON_ERR_WORKSPACE, MUON_ERR_CUDA, MUON_ERR_TIMEOUT = range(6)
+
+def lib_path() -> str:
+    return CHECKED_LIB_PATH if os.environ.get("AURORA_MUON_CHECKED", "0") == "1" else LIB_PATH
+
+(MUON_OK, MUON_ERR_INVALID_ARG, MUON_ERR_UNSUPPORTED, MUON_ERR_WORKSPACE, MUON_ERR_CUDA, MUON_ERR_TIMEOUT,
+ MUON_ERR_BOUNDS) = range(7)
 MUON_F32, MUON_BF16 = 0, 1
 MUON_GEMM_BF16, MUON_GEMM_FP32, MUON_GEMM_BF16_SIMT = 0, 1, 2
 
 EXPORTS = ["muon_config_default", "muon_workspace_size", "muon_step", "ns_polar", "aurora_polar",
            "opnorm_normalize", "uw_floor_apply", "muon_last_device_status", "muon_status_string",
            "muon_profile_enable", "muon_profile_read", "opnorm_normalize_noalloc",
-           "adamw_config_default", "adamw_step", "muon_selftest_wait_timeout"]
+           "adamw_config_default", "adamw_step", "muon_selftest_wait_timeout", "muon_build_checked",
+           "muon_last_check_line", "muon_selftest_bounds_check"]
 
 
 class MuonShape(C.Structure):
@@ -68,10 +77,11 @@ def load():
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with "
+    path = lib_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
                           "`python -m aurora_orthogonalised_optimizer_b200.build`")
-    lib = C.CDLL(LIB_PATH)
+    lib = C.CDLL(path)
     P = C.c_void_p
     PP = C.POINTER(C.c_void_p)
     lib.muon_config_default.argtypes = [C.POINTER(MuonConfig)]
@@ -98,6 +108,12 @@ def load():
     lib.muon_selftest_wait_timeout.restype = C.c_int
     lib.muon_last_device_status.argtypes = [P]
     lib.muon_last_device_status.restype = C.c_int
+    lib.muon_build_checked.argtypes = []
+    lib.muon_build_checked.restype = C.c_int
+    lib.muon_last_check_line.argtypes = []
+    lib.muon_last_check_line.restype = C.c_int
+    lib.muon_selftest_bounds_check.argtypes = [P]
+    lib.muon_selftest_bounds_check.restype = C.c_int
     lib.muon_status_string.argtypes = [C.c_int]
     lib.muon_status_string.restype = C.c_char_p
     lib.adamw_config_default.argtypes = [C.POINTER(AdamWConfig)]
@@ -300,6 +316,21 @@ def selftest_wait_timeout(max_cycles: int = 1_000_000, stream=None) -> int:
 
 def last_device_status(stream=None) -> int:
     return int(load().muon_last_device_status(_stream(stream)))
+
+
+def build_checked() -> bool:
+    """True when the loaded library is the bounds-checked build."""
+    return bool(load().muon_build_checked())
+
+
+def last_check_line() -> int:
+    """Source line of the first failed index test (checked build), 0 if none."""
+    return int(load().muon_last_check_line())
+
+
+def selftest_bounds_check(stream=None) -> int:
+    """Launch the index-test self-test (see the header)."""
+    return int(load().muon_selftest_bounds_check(_stream(stream)))
 
 
 def profile_enable(on: bool = True) -> None:

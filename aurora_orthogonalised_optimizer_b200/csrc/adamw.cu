@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(kAwThreads) k_adamw(const AwTable T) {
     const int64_t j = base + 8 * (threadIdx.x + kAwThreads * k);
     const int64_t left = d.numel - j;
     cnt[k] = left <= 0 ? 0 : (left >= 8 ? 8 : (int)left);
+    if (cnt[k] > 0 && !AM_IN(j, cnt[k], d.numel)) cnt[k] = 0;
     if (cnt[k] == 8) {
       ld8(d.p, j, T.param_dtype, p[k]);
       ld8(d.g, j, T.grad_dtype, g[k]);
@@ -119,6 +120,9 @@ int aw_iters() {
 }
 
 }  // namespace
+
+AM_CHECK_READER(read_and_clear_check_adamw)
+
 }  // namespace am
 
 using namespace am;

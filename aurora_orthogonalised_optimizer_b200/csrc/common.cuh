@@ -80,6 +80,79 @@ __device__ __forceinline__ void st8r(void* p, int64_t row_off, int64_t j, int64_
   else st8m(p, row_off + j, dt, (int)(n - j < 8 ? (n - j > 0 ? n - j : 0) : 8), v);
 }
 
+// ---------------------------------------------------------------- checked build
+// Built with AURORA_MUON_CHECKED (build.py --checked -> libaurora_muon_checked.so),
+// every global access of the streaming, power-iteration and GEMM-epilogue
+// kernels first tests its element range [first, first + count) against the
+// extent of the buffer it addresses.  A failed test records the source line
+// in this file's sticky check word (first failure wins) and the access is
+// skipped (loads read zeros), so nothing outside a buffer is touched; the
+// host reads the words through muon_last_device_status (MUON_ERR_BOUNDS).
+// In the normal build the test is the constant true and compiles away.
+#ifdef AURORA_MUON_CHECKED
+static __device__ unsigned int g_check_line = 0;
+__device__ __noinline__ inline void check_fail(unsigned int line) { atomicCAS(&g_check_line, 0u, line); }
+__device__ __forceinline__ bool in_range(int64_t first, int64_t count, int64_t extent, unsigned int line) {
+  if (first >= 0 && count >= 0 && first + count <= extent) return true;
+  check_fail(line);
+  return false;
+}
+#define AM_IN(first, count, extent) ::am::in_range((int64_t)(first), (int64_t)(count), (int64_t)(extent), __LINE__)
+// Host: read and clear this file's check word (current device).
+#define AM_CHECK_READER(fn)                                                        \
+  cudaError_t fn(unsigned int* out) {                                              \
+    unsigned int v = 0, zero = 0;                                                  \
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_check_line, sizeof(v));             \
+    if (e != cudaSuccess) return e;                                                \
+    *out = v;                                                                      \
+    return v ? cudaMemcpyToSymbol(g_check_line, &zero, sizeof(zero)) : cudaSuccess; \
+  }
+#else
+#define AM_IN(first, count, extent) true
+#define AM_CHECK_READER(fn)             \
+  cudaError_t fn(unsigned int* out) {   \
+    *out = 0;                           \
+    return cudaSuccess;                 \
+  }
+#endif
+// Elements of the 8-group at column j of a row of length n (0 to 8).
+__device__ __forceinline__ int64_t cnt8(int64_t n, int64_t j) { return n - j >= 8 ? 8 : (n - j > 0 ? n - j : 0); }
+// Extents of the per-matrix buffers (elements).
+#define AM_EXT_ORIG(d) ((d).m * (d).n)                 /* W, G, M, V */
+#define AM_EXT_X(d) ((d).s * (d).ldl)                  /* uX, UX, X0 */
+#define AM_EXT_VEC(d) ((((d).l > (d).s ? (d).l : (d).s) + 63) / 64 * 64)   /* vec0, vec1 */
+
+// Checked forms of the access helpers: `ext` is the extent (elements) of the
+// buffer p points to.  A range outside it is skipped (a load gives zeros).
+#define ld8c(ext, p, i, dt, v)                                  \
+  do {                                                          \
+    if (AM_IN((i), 8, (ext))) ::am::ld8((p), (i), (dt), (v));   \
+    else for (int _q = 0; _q < 8; ++_q) (v)[_q] = 0.f;          \
+  } while (0)
+#define st8c(ext, p, i, dt, v)                                  \
+  do {                                                          \
+    if (AM_IN((i), 8, (ext))) ::am::st8((p), (i), (dt), (v));   \
+  } while (0)
+#define ld8rc(ext, p, row_off, j, n, vec, dt, v)                                        \
+  do {                                                                                  \
+    if (AM_IN((row_off) + (j), ::am::cnt8((n), (j)), (ext)))                            \
+      ::am::ld8r((p), (row_off), (j), (n), (vec), (dt), (v));                           \
+    else for (int _q = 0; _q < 8; ++_q) (v)[_q] = 0.f;                                  \
+  } while (0)
+#define st8rc(ext, p, row_off, j, n, vec, dt, v)                                        \
+  do {                                                                                  \
+    if (AM_IN((row_off) + (j), ::am::cnt8((n), (j)), (ext)))                            \
+      ::am::st8r((p), (row_off), (j), (n), (vec), (dt), (v));                           \
+  } while (0)
+// 16 bytes (8 bf16) at element i of a bf16 buffer through the read-only path
+__device__ __forceinline__ uint4 ldg8bf(int64_t ext, const __nv_bfloat16* p, int64_t i, unsigned int line) {
+#ifdef AURORA_MUON_CHECKED
+  if (!in_range(i, 8, ext, line)) return make_uint4(0, 0, 0, 0);
+#endif
+  return __ldg(reinterpret_cast<const uint4*>(p + i));
+}
+#define LDG8BF(ext, p, i) ::am::ldg8bf((ext), (p), (i), __LINE__)
+
 // ---------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -122,10 +195,13 @@ struct MatDesc {
   float* vec1;
   float* rho_slot;    // bucket-ordered copy of rho read by the GEMM epilogues
   float* gvp;         // fused power iteration: one partial X^T z (ldl floats) per row item
+  float* colsq;       // Aurora D update: column sums of U^2 (X orientation) per 32-row block,
+                      // [ceil(s / 32)][round64(l)] floats, written by the last update GEMM
   int64_t m, n, s, l, ldl;
   int tall;           // m > n
   int idx;            // matrix index (scalar block row)
   int part;           // first partial slot of this matrix
+  int nslots;         // partial slots owned by this matrix (from part on)
   int nblk;           // blocks of this matrix in the current launch
   int flag;           // launch-specific per-matrix flag
   int gv_rows;        // fused power iteration: rows of X per item

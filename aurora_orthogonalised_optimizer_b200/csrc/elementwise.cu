@@ -60,14 +60,14 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
     float g0[8], g1[8], m0[8], m1[8], w0[8], w1[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) g0[e] = g1[e] = m0[e] = m1[e] = w0[e] = w1[e] = 0.f;
-    if (in0) ld8r(d.G, ro0, j, d.n, vec, t.grad_dtype, g0);
-    if (in1) ld8r(d.G, ro1, j, d.n, vec, t.grad_dtype, g1);
+    if (in0) ld8rc(AM_EXT_ORIG(d), d.G, ro0, j, d.n, vec, t.grad_dtype, g0);
+    if (in1) ld8rc(AM_EXT_ORIG(d), d.G, ro1, j, d.n, vec, t.grad_dtype, g1);
     if (mode == 0) {
-      if (in0) ld8r(d.M, ro0, j, d.n, vec, kF32, m0);
-      if (in1) ld8r(d.M, ro1, j, d.n, vec, kF32, m1);
+      if (in0) ld8rc(AM_EXT_ORIG(d), d.M, ro0, j, d.n, vec, kF32, m0);
+      if (in1) ld8rc(AM_EXT_ORIG(d), d.M, ro1, j, d.n, vec, kF32, m1);
       if (want_w2) {
-        if (in0) ld8r(d.W, ro0, j, d.n, vec, t.param_dtype, w0);
-        if (in1) ld8r(d.W, ro1, j, d.n, vec, t.param_dtype, w1);
+        if (in0) ld8rc(AM_EXT_ORIG(d), d.W, ro0, j, d.n, vec, t.param_dtype, w0);
+        if (in1) ld8rc(AM_EXT_ORIG(d), d.W, ro1, j, d.n, vec, t.param_dtype, w1);
       }
     }
     float su2 = 0.f, sw2 = 0.f;
@@ -87,12 +87,12 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
       sw2 += w0[e] * w0[e] + w1[e] * w1[e];
     }
     if (mode == 0) {
-      if (in0) st8r(d.M, ro0, j, d.n, vec, kF32, m0);
-      if (in1) st8r(d.M, ro1, j, d.n, vec, kF32, m1);
+      if (in0) st8rc(AM_EXT_ORIG(d), d.M, ro0, j, d.n, vec, kF32, m0);
+      if (in1) st8rc(AM_EXT_ORIG(d), d.M, ro1, j, d.n, vec, kF32, m1);
     }
     if (!d.tall) {
-      if (in0) st8r(d.uX, (r0 + rg) * d.ldl, j, d.n, xvec, t.ns_dtype, u0);
-      if (in1) st8r(d.uX, (r0 + rg + 32) * d.ldl, j, d.n, xvec, t.ns_dtype, u1);
+      if (in0) st8rc(AM_EXT_X(d), d.uX, (r0 + rg) * d.ldl, j, d.n, xvec, t.ns_dtype, u0);
+      if (in1) st8rc(AM_EXT_X(d), d.uX, (r0 + rg + 32) * d.ldl, j, d.n, xvec, t.ns_dtype, u1);
     } else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -109,11 +109,11 @@ k_prologue(const MatTable t, int mode, float mu, int nesterov, int want_w2, doub
           float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = tile[8 * cg + e][xr];
-          st8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, v);
+          st8rc(AM_EXT_X(d), d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, v);
         }
       }
     }
-    warp_partials(partials, d.part + b, 2, su2, sw2);
+    if (AM_IN(b, 1, d.nslots)) warp_partials(partials, d.part + b, 2, su2, sw2);
   }
 }
 
@@ -127,7 +127,8 @@ __global__ void k_finalize_sums(const MatTable t, const double* partials, int nq
     const int slot = q == 0 ? slot0 : slot1;
     double s = 0.0;
     const int64_t n = (int64_t)d.nblk * kWarps;
-    for (int64_t k = threadIdx.x; k < n; k += blockDim.x) s += partials[((int64_t)d.part * kWarps + k) * nq + q];
+    for (int64_t k = threadIdx.x; k < n; k += blockDim.x)
+      if (AM_IN(k, 1, (int64_t)d.nslots * kWarps)) s += partials[((int64_t)d.part * kWarps + k) * nq + q];
     s = block_sum(s, red);
     if (threadIdx.x == 0 && slot >= 0) scal[d.idx * S_COUNT + slot] = s;
   }
@@ -157,7 +158,7 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
 #pragma unroll 4
     for (int64_t i = w; i < d.s; i += kWarps) {
       float x[8];
-      ld8r(X, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+      ld8rc(AM_EXT_X(d), X, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += x[e] * x[e];
     }
@@ -170,6 +171,7 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
     float sum = 0.f;
 #pragma unroll
     for (int r = 0; r < kWarps; ++r) sum += part[r][threadIdx.x];
+    if (!AM_IN(jj, 1, d.l)) return;
     if (mode == 0) {
       d.D[jj] = 1.f / fmaxf(sqrtf(sum), pp_eps);
     } else {
@@ -177,6 +179,65 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
       const float target = (float)d.s / (float)d.l;
       d.D[jj] = d.D[jj] * powf(target / row_sq, beta);
     }
+  }
+}
+
+// Column sums of squares of uX over 32-row blocks, into MatDesc::colsq
+// ([ceil(s / 32)][round64(l)] floats): a block covers 256 rows x 256 columns,
+// warp w rows 32 w .. +31 of them, each lane 8 columns (one 16-byte load per
+// row).  Many short independent blocks instead of one block walking every
+// row of a column strip.
+__global__ void __launch_bounds__(kEwThreads)
+k_colsq_partial(const MatTable t) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t strips = (d.l + kColStrip - 1) / kColStrip;
+  const int64_t b = blockIdx.x - t.blk_prefix[mi];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t rb = (b / strips) * 8 + w;                  // 32-row block of this warp
+  const int64_t j = (b % strips) * kColStrip + 8 * lane;
+  const int64_t i0 = rb * 32;
+  if (i0 >= d.s || j >= d.l) return;
+  const int64_t i1 = min(d.s, i0 + 32);
+  const bool vec = (d.ldl & 7) == 0;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+  for (int64_t i = i0; i < i1; ++i) {
+    float x[8];
+    ld8rc(AM_EXT_X(d), d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += x[e] * x[e];
+  }
+  float* q = d.colsq + rb * ((d.l + 63) / 64 * 64) + j;     // j + 8 <= round64(l)
+  if (!AM_IN(rb * ((d.l + 63) / 64 * 64) + j, 8, ((d.s + 31) / 32) * ((d.l + 63) / 64 * 64))) return;
+  reinterpret_cast<float4*>(q)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  reinterpret_cast<float4*>(q)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// Aurora D from the partial column sums in MatDesc::colsq (written per
+// 32-row block by k_colsq_partial from uX, or by the last update GEMM of the
+// previous polar from U): one thread per column sums the ceil(s / 32)
+// partials in block order (deterministic).
+//   mode 0 (D init):  D_j = 1 / max(sqrt(sum), pp_eps)
+//   mode 1 (D update): D_j *= (target / max(sum, pp_eps^2))^beta, target = s / l
+__global__ void __launch_bounds__(kColStrip)
+k_colsq_update(const MatTable t, int mode, float pp_eps, float beta) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t j = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kColStrip + threadIdx.x;
+  if (j >= d.l) return;
+  const int64_t nb = (d.s + 31) / 32, ldq = (d.l + 63) / 64 * 64;
+  const float* q = d.colsq + j;
+  float sum = 0.f;
+  for (int64_t b = 0; b < nb; ++b)
+    if (AM_IN(b * ldq + j, 1, nb * ldq)) sum += q[b * ldq];
+  if (!AM_IN(j, 1, d.l)) return;
+  if (mode == 0) {
+    d.D[j] = 1.f / fmaxf(sqrtf(sum), pp_eps);
+  } else {
+    const float row_sq = fmaxf(sum, pp_eps * pp_eps);
+    const float target = (float)d.s / (float)d.l;
+    d.D[j] = d.D[j] * powf(target / row_sq, beta);
   }
 }
 
@@ -199,19 +260,19 @@ k_scale_cols(const MatTable t, double* partials) {
       const bool in0 = r0 + rg < d.s, in1 = r0 + rg + 32 < d.s;
       const int64_t ro0 = (r0 + rg) * d.ldl, ro1 = (r0 + rg + 32) * d.ldl;
       float dj[8], x0[8], x1[8];
-      ld8r(d.D, 0, j, d.l, true, kF32, dj);
-      if (in0) ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, x0);
-      if (in1) ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, x1);
+      ld8rc(d.l, d.D, 0, j, d.l, true, kF32, dj);
+      if (in0) ld8rc(AM_EXT_X(d), d.uX, ro0, j, d.l, vec, t.ns_dtype, x0);
+      if (in1) ld8rc(AM_EXT_X(d), d.uX, ro1, j, d.l, vec, t.ns_dtype, x1);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         x0[e] = in0 ? x0[e] * dj[e] : 0.f;
         x1[e] = in1 ? x1[e] * dj[e] : 0.f;
         s2 += x0[e] * x0[e] + x1[e] * x1[e];
       }
-      if (in0) st8r(d.X0, ro0, j, d.l, vec, t.ns_dtype, x0);
-      if (in1) st8r(d.X0, ro1, j, d.l, vec, t.ns_dtype, x1);
+      if (in0) st8rc(AM_EXT_X(d), d.X0, ro0, j, d.l, vec, t.ns_dtype, x0);
+      if (in1) st8rc(AM_EXT_X(d), d.X0, ro1, j, d.l, vec, t.ns_dtype, x1);
     }
-    warp_partials(partials, d.part + b, 1, s2, 0.f);
+    if (AM_IN(b, 1, d.nslots)) warp_partials(partials, d.part + b, 1, s2, 0.f);
   }
 }
 
@@ -302,12 +363,12 @@ k_matvec(const MatTable t, int dir) {
 #pragma unroll 2
       for (int64_t j = 8 * lane; j < d.l; j += 256) {
         float v[8];
-        ld8r(in, 0, j, d.l, true, kF32, v);
+        ld8rc(AM_EXT_VEC(d), in, 0, j, d.l, true, kF32, v);
 #pragma unroll
         for (int r = 0; r < kMatvecRowsPerWarp; ++r) {
           if (i0 + r < d.s) {
             float x[8];
-            ld8r(d.uX, (i0 + r) * d.ldl, j, d.l, vec, t.ns_dtype, x);
+            ld8rc(AM_EXT_X(d), d.uX, (i0 + r) * d.ldl, j, d.l, vec, t.ns_dtype, x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[r] += x[e] * v[e];
           }
@@ -316,7 +377,7 @@ k_matvec(const MatTable t, int dir) {
 #pragma unroll
       for (int r = 0; r < kMatvecRowsPerWarp; ++r) {
         const float a = warp_sum(acc[r]);
-        if (lane == 0 && i0 + r < d.s) out[i0 + r] = a;
+        if (lane == 0 && i0 + r < d.s && AM_IN(i0 + r, 1, AM_EXT_VEC(d))) out[i0 + r] = a;
       }
     }
   } else {
@@ -329,8 +390,8 @@ k_matvec(const MatTable t, int dir) {
 #pragma unroll 4
       for (int64_t i = rl; i < d.s; i += 32) {
         float x[8];
-        ld8r(d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
-        const float y = in[i];
+        ld8rc(AM_EXT_X(d), d.uX, i * d.ldl, j, d.l, vec, t.ns_dtype, x);
+        const float y = AM_IN(i, 1, AM_EXT_VEC(d)) ? in[i] : 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] += x[e] * y;
       }
@@ -340,7 +401,7 @@ k_matvec(const MatTable t, int dir) {
     __syncthreads();
     if (threadIdx.x < kColDotStrip) {
       const int64_t jj = (int64_t)b * kColDotStrip + threadIdx.x;
-      if (jj < d.l) {
+      if (jj < d.l && AM_IN(jj, 1, AM_EXT_VEC(d))) {
         float sum = 0.f;
         for (int r = 0; r < 32; ++r) sum += part[r][threadIdx.x];
         out[jj] = sum;
@@ -398,15 +459,15 @@ k_dots(const MatTable t, double* partials) {
       float U0[8], u0[8], U1[8], u1[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) U0[e] = u0[e] = U1[e] = u1[e] = 0.f;
-      if (in0) { ld8r(d.UX, ro0, j, d.l, vec, t.ns_dtype, U0); ld8r(d.uX, ro0, j, d.l, vec, t.ns_dtype, u0); }
-      if (in1) { ld8r(d.UX, ro1, j, d.l, vec, t.ns_dtype, U1); ld8r(d.uX, ro1, j, d.l, vec, t.ns_dtype, u1); }
+      if (in0) { ld8rc(AM_EXT_X(d), d.UX, ro0, j, d.l, vec, t.ns_dtype, U0); ld8rc(AM_EXT_X(d), d.uX, ro0, j, d.l, vec, t.ns_dtype, u0); }
+      if (in1) { ld8rc(AM_EXT_X(d), d.UX, ro1, j, d.l, vec, t.ns_dtype, U1); ld8rc(AM_EXT_X(d), d.uX, ro1, j, d.l, vec, t.ns_dtype, u1); }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         a += U0[e] * U0[e] + U1[e] * U1[e];
         c += U0[e] * u0[e] + U1[e] * u1[e];
       }
     }
-    warp_partials(partials, d.part + b, 2, a, c);
+    if (AM_IN(b, 1, d.nslots)) warp_partials(partials, d.part + b, 2, a, c);
   }
 }
 
@@ -443,7 +504,7 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
       in[k] = i < d.m && j < d.n;
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[k][e] = w[k][e] = 0.f;
-      if (in[k] && update_w) ld8r(d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
+      if (in[k] && update_w) ld8rc(AM_EXT_ORIG(d), d.W, i * d.n, j, d.n, vec, t.param_dtype, w[k]);
     }
     if (d.tall) {
       // V = cU U + cu u is formed in the X orientation (X tile rows = original
@@ -456,8 +517,8 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) xU[e] = xu[e] = 0.f;
         if (xi < d.n && xj < d.m) {
-          if (need_U) ld8r(d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xU);
-          if (need_u) ld8r(d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xu);
+          if (need_U) ld8rc(AM_EXT_X(d), d.UX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xU);
+          if (need_u) ld8rc(AM_EXT_X(d), d.uX, xi * d.ldl, xj, d.m, xvec, t.ns_dtype, xu);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) tV[rg + 32 * k][8 * cg + e] = cU * xU[e] + cu * xu[e];
@@ -475,8 +536,8 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
         float U[8], u[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) U[e] = u[e] = 0.f;
-        if (need_U) ld8r(d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U);
-        if (need_u) ld8r(d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
+        if (need_U) ld8rc(AM_EXT_X(d), d.UX, i * d.ldl, j, d.n, xvec, t.ns_dtype, U);
+        if (need_u) ld8rc(AM_EXT_X(d), d.uX, i * d.ldl, j, d.n, xvec, t.ns_dtype, u);
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[k][e] = cU * U[e] + cu * u[e];
       }
@@ -487,8 +548,8 @@ k_epilogue(const MatTable t, float lr, int update_w, const double* scal) {
       const int64_t ro = (r0 + rg + 32 * k) * d.n;
 #pragma unroll
       for (int e = 0; e < 8; ++e) w[k][e] -= lr * v[k][e];
-      if (d.V) st8r(d.V, ro, j, d.n, vec, kF32, v[k]);
-      if (update_w) st8r(d.W, ro, j, d.n, vec, t.param_dtype, w[k]);
+      if (d.V) st8rc(AM_EXT_ORIG(d), d.V, ro, j, d.n, vec, kF32, v[k]);
+      if (update_w) st8rc(AM_EXT_ORIG(d), d.W, ro, j, d.n, vec, t.param_dtype, w[k]);
     }
   }
 }
@@ -529,9 +590,9 @@ k_epilogue_tall_bf16(const MatTable t, float lr, int update_w, const double* sca
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int64_t i = r0 + rg + 32 * k, xi = c0 + rg + 32 * k;
-      w[k] = update_w ? __ldg(reinterpret_cast<const uint4*>(W + i * d.n + c0 + 8 * cg)) : make_uint4(0, 0, 0, 0);
-      xU[k] = need_U ? __ldg(reinterpret_cast<const uint4*>(UX + xi * d.ldl + r0 + 8 * cg)) : make_uint4(0, 0, 0, 0);
-      xu[k] = need_u ? __ldg(reinterpret_cast<const uint4*>(uX + xi * d.ldl + r0 + 8 * cg)) : make_uint4(0, 0, 0, 0);
+      w[k] = update_w ? LDG8BF(AM_EXT_ORIG(d), W, i * d.n + c0 + 8 * cg) : make_uint4(0, 0, 0, 0);
+      xU[k] = need_U ? LDG8BF(AM_EXT_X(d), UX, xi * d.ldl + r0 + 8 * cg) : make_uint4(0, 0, 0, 0);
+      xu[k] = need_u ? LDG8BF(AM_EXT_X(d), uX, xi * d.ldl + r0 + 8 * cg) : make_uint4(0, 0, 0, 0);
     }
   };
   auto process = [&](int b, int buf, const uint4 (&w)[2], const uint4 (&xU)[2], const uint4 (&xu)[2]) {
@@ -551,12 +612,12 @@ k_epilogue_tall_bf16(const MatTable t, float lr, int update_w, const double* sca
       float v[8], wf[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = tV[buf][8 * cg + e][rg + 32 * k];
-      if (d.V) st8(d.V, ro, kF32, v);
+      if (d.V) st8c(AM_EXT_ORIG(d), d.V, ro, kF32, v);
       if (update_w) {
         bf16x8_to_f32(w[k], wf);
 #pragma unroll
         for (int e = 0; e < 8; ++e) wf[e] -= lr * v[e];
-        st8(d.W, ro, kBF16, wf);
+        st8c(AM_EXT_ORIG(d), d.W, ro, kBF16, wf);
       }
     }
   };
@@ -596,10 +657,10 @@ k_prologue_flat(const MatTable t, int mode, float mu, int nesterov, int want_w2,
 #pragma unroll
       for (int q = 0; q < 8; ++q) g[k][q] = m[k][q] = w[k][q] = 0.f;
       if (!in[k]) continue;
-      ld8(d.G, e, t.grad_dtype, g[k]);
+      ld8c(AM_EXT_ORIG(d), d.G, e, t.grad_dtype, g[k]);
       if (mode == 0) {
-        ld8(d.M, e, kF32, m[k]);
-        if (want_w2) ld8(d.W, e, t.param_dtype, w[k]);
+        ld8c(AM_EXT_ORIG(d), d.M, e, kF32, m[k]);
+        if (want_w2) ld8c(AM_EXT_ORIG(d), d.W, e, t.param_dtype, w[k]);
       }
     }
 #pragma unroll
@@ -618,10 +679,10 @@ k_prologue_flat(const MatTable t, int mode, float mu, int nesterov, int want_w2,
         su2 += u[q] * u[q];
         sw2 += w[k][q] * w[k][q];
       }
-      if (mode == 0) st8(d.M, e, kF32, m[k]);
-      st8(d.uX, e, t.ns_dtype, u);
+      if (mode == 0) st8c(AM_EXT_ORIG(d), d.M, e, kF32, m[k]);
+      st8c(AM_EXT_X(d), d.uX, e, t.ns_dtype, u);
     }
-    warp_partials(partials, d.part + c, 2, su2, sw2);
+    if (AM_IN(c, 1, d.nslots)) warp_partials(partials, d.part + c, 2, su2, sw2);
   }
 }
 
@@ -631,6 +692,11 @@ k_scale_cols_flat(const MatTable t, double* partials) {
   const MatDesc& d = t.mats[mi];
   const int64_t total = d.s * d.l;
   const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
+  // column of each of this thread's two 8-groups, advanced chunk by chunk
+  // (one division per block instead of one per group)
+  const int64_t step = kFlatChunk % d.l;
+  int64_t col[2] = {(c0 * kFlatChunk + 8 * threadIdx.x) % d.l,
+                    (c0 * kFlatChunk + 8 * (threadIdx.x + kEwThreads)) % d.l};
   for (int64_t c = c0; c < c0 + kEwTilesPerCta && c * kFlatChunk < total; ++c) {
     float s2 = 0.f;
     float x[2][8], dj[2][8];
@@ -639,9 +705,12 @@ k_scale_cols_flat(const MatTable t, double* partials) {
     for (int k = 0; k < 2; ++k) {
       const int64_t e = c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k);
       in[k] = e < total;
-      if (!in[k]) continue;
-      ld8(d.uX, e, t.ns_dtype, x[k]);
-      ld8(d.D, e % d.l, kF32, dj[k]);
+      if (in[k]) {
+        ld8c(AM_EXT_X(d), d.uX, e, t.ns_dtype, x[k]);
+        ld8c(d.l, d.D, col[k], kF32, dj[k]);
+      }
+      col[k] += step;
+      if (col[k] >= d.l) col[k] -= d.l;
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -652,9 +721,9 @@ k_scale_cols_flat(const MatTable t, double* partials) {
         x[k][q] *= dj[k][q];
         s2 += x[k][q] * x[k][q];
       }
-      st8(d.X0, e, t.ns_dtype, x[k]);
+      st8c(AM_EXT_X(d), d.X0, e, t.ns_dtype, x[k]);
     }
-    warp_partials(partials, d.part + c, 1, s2, 0.f);
+    if (AM_IN(c, 1, d.nslots)) warp_partials(partials, d.part + c, 1, s2, 0.f);
   }
 }
 
@@ -669,19 +738,30 @@ k_scale_cols_flat_bf16(const MatTable t, double* partials) {
   const int64_t c1 = min(c0 + kEwTilesPerCta, (total + kFlatChunk - 1) / kFlatChunk);
   const __nv_bfloat16* uX = reinterpret_cast<const __nv_bfloat16*>(d.uX);
   auto off = [&](int64_t c, int k) { return c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k); };
+  // column of each of this thread's two 8-groups in the chunk load() fetches
+  // next: chunks are loaded in order, so it advances by kFlatChunk mod l
+  // (one division per block instead of one per group)
+  const int64_t step = kFlatChunk % d.l;
+  int64_t col[2] = {off(c0, 0) % d.l, off(c0, 1) % d.l};
   auto load = [&](int64_t c, uint4 (&x)[2], float4 (&dj)[2][2]) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int64_t e = off(c, k);
       if (e < total) {
-        x[k] = __ldg(reinterpret_cast<const uint4*>(uX + e));
-        const float4* dp = reinterpret_cast<const float4*>(d.D + e % d.l);
-        dj[k][0] = __ldg(dp);
-        dj[k][1] = __ldg(dp + 1);
+        x[k] = LDG8BF(AM_EXT_X(d), uX, e);
+        const float4* dp = reinterpret_cast<const float4*>(d.D + col[k]);
+        if (AM_IN(col[k], 8, d.l)) {
+          dj[k][0] = __ldg(dp);
+          dj[k][1] = __ldg(dp + 1);
+        } else {
+          dj[k][0] = dj[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       } else {
         x[k] = make_uint4(0, 0, 0, 0);
         dj[k][0] = dj[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      col[k] += step;
+      if (col[k] >= d.l) col[k] -= d.l;
     }
   };
   auto process = [&](int64_t c, const uint4 (&x)[2], const float4 (&dj)[2][2]) {
@@ -699,9 +779,9 @@ k_scale_cols_flat_bf16(const MatTable t, double* partials) {
         v[q] *= dd[q];
         s2 += v[q] * v[q];
       }
-      st8(d.X0, e, kBF16, v);
+      st8c(AM_EXT_X(d), d.X0, e, kBF16, v);
     }
-    warp_partials(partials, d.part + c, 1, s2, 0.f);
+    if (AM_IN(c, 1, d.nslots)) warp_partials(partials, d.part + c, 1, s2, 0.f);
   };
   if (c0 >= c1) return;
   uint4 xa[2], xb[2];
@@ -731,8 +811,8 @@ k_dots_flat(const MatTable t, double* partials) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) U[k][q] = u[k][q] = 0.f;
       if (e < total) {
-        ld8(d.UX, e, t.ns_dtype, U[k]);
-        ld8(d.uX, e, t.ns_dtype, u[k]);
+        ld8c(AM_EXT_X(d), d.UX, e, t.ns_dtype, U[k]);
+        ld8c(AM_EXT_X(d), d.uX, e, t.ns_dtype, u[k]);
       }
     }
 #pragma unroll
@@ -742,7 +822,7 @@ k_dots_flat(const MatTable t, double* partials) {
         a += U[k][q] * U[k][q];
         cc += U[k][q] * u[k][q];
       }
-    warp_partials(partials, d.part + c, 2, a, cc);
+    if (AM_IN(c, 1, d.nslots)) warp_partials(partials, d.part + c, 2, a, cc);
   }
 }
 
@@ -765,9 +845,9 @@ k_epilogue_flat(const MatTable t, float lr, int update_w, const double* scal) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) U[k][q] = u[k][q] = w[k][q] = 0.f;
       if (!in[k]) continue;
-      if (need_U) ld8(d.UX, e, t.ns_dtype, U[k]);
-      if (need_u) ld8(d.uX, e, t.ns_dtype, u[k]);
-      if (update_w) ld8(d.W, e, t.param_dtype, w[k]);
+      if (need_U) ld8c(AM_EXT_X(d), d.UX, e, t.ns_dtype, U[k]);
+      if (need_u) ld8c(AM_EXT_X(d), d.uX, e, t.ns_dtype, u[k]);
+      if (update_w) ld8c(AM_EXT_ORIG(d), d.W, e, t.param_dtype, w[k]);
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -779,8 +859,8 @@ k_epilogue_flat(const MatTable t, float lr, int update_w, const double* scal) {
         v[q] = cU * U[k][q] + cu * u[k][q];
         w[k][q] -= lr * v[q];
       }
-      if (d.V) st8(d.V, e, kF32, v);
-      if (update_w) st8(d.W, e, t.param_dtype, w[k]);
+      if (d.V) st8c(AM_EXT_ORIG(d), d.V, e, kF32, v);
+      if (update_w) st8c(AM_EXT_ORIG(d), d.W, e, t.param_dtype, w[k]);
     }
   }
 }
@@ -807,10 +887,14 @@ k_prologue_tall_bf16(const MatTable t, float mu, int nesterov, int want_w2, doub
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int64_t e = (r0 + rg + 32 * k) * d.n + c0 + 8 * cg;
-      r.g[k] = __ldg(reinterpret_cast<const uint4*>(G + e));
-      r.m[k][0] = reinterpret_cast<const float4*>(d.M + e)[0];
-      r.m[k][1] = reinterpret_cast<const float4*>(d.M + e)[1];
-      r.w[k] = want_w2 ? __ldg(reinterpret_cast<const uint4*>(W + e)) : make_uint4(0, 0, 0, 0);
+      r.g[k] = LDG8BF(AM_EXT_ORIG(d), G, e);
+      if (AM_IN(e, 8, AM_EXT_ORIG(d))) {
+        r.m[k][0] = reinterpret_cast<const float4*>(d.M + e)[0];
+        r.m[k][1] = reinterpret_cast<const float4*>(d.M + e)[1];
+      } else {
+        r.m[k][0] = r.m[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      r.w[k] = want_w2 ? LDG8BF(AM_EXT_ORIG(d), W, e) : make_uint4(0, 0, 0, 0);
     }
   };
   auto process = [&](int b, int buf, const Raw& r) {
@@ -836,7 +920,7 @@ k_prologue_tall_bf16(const MatTable t, float mu, int nesterov, int want_w2, doub
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      st8(d.M, (r0 + rg + 32 * k) * d.n + c0 + 8 * cg, kF32, m[k]);
+      st8c(AM_EXT_ORIG(d), d.M, (r0 + rg + 32 * k) * d.n + c0 + 8 * cg, kF32, m[k]);
 #pragma unroll
       for (int e = 0; e < 8; ++e) tile[buf][rg + 32 * k][8 * cg + e] = u[k][e];
     }
@@ -848,9 +932,9 @@ k_prologue_tall_bf16(const MatTable t, float mu, int nesterov, int want_w2, doub
       float v[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = tile[buf][8 * cg + e][xr];
-      st8(d.uX, (c0 + xr) * d.ldl + r0 + 8 * cg, kBF16, v);
+      st8c(AM_EXT_X(d), d.uX, (c0 + xr) * d.ldl + r0 + 8 * cg, kBF16, v);
     }
-    warp_partials(partials, d.part + b, 2, su2, sw2);
+    if (AM_IN(b, 1, d.nslots)) warp_partials(partials, d.part + b, 2, su2, sw2);
   };
   if (b0 >= b1) return;
   Raw ra, rb;
@@ -887,9 +971,9 @@ k_epilogue_flat_bf16(const MatTable t, float lr, int update_w, const double* sca
     for (int k = 0; k < 2; ++k) {
       const int64_t e = off(c, k);
       const bool in = e < total;
-      a[k] = in && need_U ? __ldg(reinterpret_cast<const uint4*>(UX + e)) : z4;
-      b[k] = in && need_u ? __ldg(reinterpret_cast<const uint4*>(uX + e)) : z4;
-      w[k] = in && update_w ? __ldg(reinterpret_cast<const uint4*>(W + e)) : z4;
+      a[k] = in && need_U ? LDG8BF(AM_EXT_X(d), UX, e) : z4;
+      b[k] = in && need_u ? LDG8BF(AM_EXT_X(d), uX, e) : z4;
+      w[k] = in && update_w ? LDG8BF(AM_EXT_ORIG(d), W, e) : z4;
     }
   };
   auto process = [&](int64_t c, const uint4 (&a)[2], const uint4 (&b)[2], const uint4 (&w)[2]) {
@@ -906,8 +990,8 @@ k_epilogue_flat_bf16(const MatTable t, float lr, int update_w, const double* sca
         v[q] = cU * U[q] + cu * u[q];
         wf[q] -= lr * v[q];
       }
-      if (d.V) st8(d.V, e, kF32, v);
-      if (update_w) st8(d.W, e, kBF16, wf);
+      if (d.V) st8c(AM_EXT_ORIG(d), d.V, e, kF32, v);
+      if (update_w) st8c(AM_EXT_ORIG(d), d.W, e, kBF16, wf);
     }
   };
   if (c0 >= c1) return;
@@ -939,8 +1023,8 @@ k_sumsq_wv(const MatTable t, double* partials) {
     const int64_t e0 = (int64_t)b * 4096 + 8 * (threadIdx.x + 256 * k);
     if (e0 < total) {
       float w[8], v[8];
-      ld8r(d.W, 0, e0, total, true, t.param_dtype, w);
-      ld8r(d.V, 0, e0, total, true, kF32, v);
+      ld8rc(AM_EXT_ORIG(d), d.W, 0, e0, total, true, t.param_dtype, w);
+      ld8rc(AM_EXT_ORIG(d), d.V, 0, e0, total, true, kF32, v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         sw += w[e] * w[e];
@@ -948,7 +1032,7 @@ k_sumsq_wv(const MatTable t, double* partials) {
       }
     }
   }
-  warp_partials(partials, d.part + b, 2, sv, sw);
+  if (AM_IN(b, 1, d.nslots)) warp_partials(partials, d.part + b, 2, sv, sw);
 }
 
 __global__ void __launch_bounds__(kEwThreads)
@@ -964,10 +1048,10 @@ k_scale_v(const MatTable t, const double* scal) {
     const int64_t e0 = (int64_t)b * 4096 + 8 * (threadIdx.x + 256 * k);
     if (e0 < total) {
       float v[8];
-      ld8r(d.V, 0, e0, total, true, kF32, v);
+      ld8rc(AM_EXT_ORIG(d), d.V, 0, e0, total, true, kF32, v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] *= c;
-      st8r(d.V, 0, e0, total, true, kF32, v);
+      st8rc(AM_EXT_ORIG(d), d.V, 0, e0, total, true, kF32, v);
     }
   }
 }
@@ -984,6 +1068,20 @@ __global__ void k_sigma_out(const MatTable t, const double* scal, float* sigma_o
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= t.count) return;
   sigma_out[t.mats[k].idx] = (float)scal[t.mats[k].idx * S_COUNT + S_SIGMA];
+}
+
+AM_CHECK_READER(read_and_clear_check_elementwise)
+
+// Tests the element range [5, 6) against an extent of 4 and touches no
+// memory: in the checked build the test fails and is recorded.
+__global__ void k_bounds_selftest() {
+  const int64_t first = 5 + (int64_t)threadIdx.x;
+  if (!AM_IN(first, 1, 4)) return;
+}
+
+cudaError_t launch_bounds_selftest(cudaStream_t st) {
+  k_bounds_selftest<<<1, 1, 0, st>>>();
+  return cudaGetLastError();
 }
 
 // ============================================================================
@@ -1027,6 +1125,16 @@ cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, 
                            cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   k_colnorm<<<nblk, kEwThreads, 0, st>>>(t, mode, pp_eps, beta);
+  return cudaGetLastError();
+}
+cudaError_t launch_colsq_partial(const MatTable& t, int nblk, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_colsq_partial<<<nblk, kEwThreads, 0, st>>>(t);
+  return cudaGetLastError();
+}
+cudaError_t launch_colsq_update(const MatTable& t, int nblk, int mode, float pp_eps, float beta, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_colsq_update<<<nblk, kColStrip, 0, st>>>(t, mode, pp_eps, beta);
   return cudaGetLastError();
 }
 cudaError_t launch_scale_cols(const MatTable& t, int nblk, double* partials, cudaStream_t st) {

@@ -45,6 +45,9 @@ struct BucketPlan {
   std::vector<int> members;
   size_t off_uX, off_P, off_Q, off_A, off_B, off_D, off_v0, off_v1, off_rho;
   size_t off_dots;       // fused <U,U>, <U,u> partials of the last update GEMM (16 doubles per tile)
+  size_t off_colsq;      // Aurora D: per 32-row block column sums of squares (uX, then U)
+  bool colsq = false;    // the bucket has that buffer
+  bool colsq_gemm = false;  // its D updates read sums the last update GEMM wrote
   int64_t dot_tiles;     // tiles per member reserved there (both tensor-core variants fit)
 };
 
@@ -129,6 +132,17 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
                              tc_tile_count(GK_UPD, (int)b.s, (int)b.l, false, &tm, &tn));
     b.off_dots = off;
     off = align_up(off + b.members.size() * (size_t)b.dot_tiles * 16 * sizeof(double));
+  }
+  // column sums of U^2 for Aurora's D update, written by the last update GEMM
+  // of each non-final polar (tensor-core mode, non-square buckets)
+  // column sums of squares per 32-row block for Aurora's D (non-square
+  // buckets): formed from uX for the D init; for the D updates, written by
+  // the last update GEMM of each non-final polar in the tensor-core mode
+  for (auto& b : p.buckets) {
+    b.colsq = cfg->aurora && b.s != b.l;
+    b.colsq_gemm = b.colsq && cfg->gemm_mode == MUON_GEMM_BF16 && cfg->pp_iterations > 1;
+    b.off_colsq = off;
+    if (b.colsq) off = align_up(off + b.members.size() * (size_t)cdiv(b.s, 32) * (size_t)round64(b.l) * sizeof(float));
   }
   p.off_scal = off;
   off = align_up(off + (size_t)n * S_COUNT * sizeof(double));
@@ -298,11 +312,14 @@ MatDesc make_desc(const Ctx& c, int i) {
   d.vec1 = wsp<float>(c, b.off_v1) + vo;
   d.rho_slot = wsp<float>(c, b.off_rho) + mp.bidx;
   d.gvp = wsp<float>(c, c.plan->off_gv) + mp.gv_off;
+  d.colsq = b.colsq ? wsp<float>(c, b.off_colsq) + (size_t)mp.bidx * (size_t)cdiv(b.s, 32) * (size_t)round64(b.l)
+                    : nullptr;
   d.gv_rows = (int)mp.gv_rows;
   d.m = mp.m; d.n = mp.n; d.s = mp.s; d.l = mp.l; d.ldl = b.ldl;
   d.tall = mp.tall;
   d.idx = i;
   d.part = (int)mp.part;
+  d.nslots = (int)std::max(cdiv(mp.m, 64) * cdiv(mp.n, 64), cdiv(mp.m * mp.n, 4096));
   return d;
 }
 
@@ -595,6 +612,14 @@ muon_status stage_newton_schulz(const Ctx& c, const std::vector<int>& bucket_ids
             g.dotu = c.ws + b.off_uX;
             g.dotp = wsp<double>(c, b.off_dots);
           }
+          if (tc && b.colsq_gemm && !final_polar[k] && it == c.cfg->ns_steps - 1) {
+            // Aurora's next D update reads these column sums instead of U, and
+            // nothing else reads this polar's U: it is not stored
+            g.colsq = wsp<float>(c, b.off_colsq);
+            g.colsq_ld = round64(b.l);
+            g.colsq_batch = cdiv(b.s, 32) * round64(b.l);
+            g.no_store = 1;
+          }
         }
         add_group(c, L, g);
         if (L.num_groups == kMaxGemmGroups) {
@@ -634,11 +659,23 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       if (e != cudaSuccess) return e;
       return launch_copy_rho(t, c.scal, c.st);
     }));
-  if (!eq_ids.empty())
-    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
-      ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
-      return launch_colnorm(t, nb, 0, pe, beta, c.st);
+  auto colsq_bytes = [](const MatTable& t) {
+    double q = 0.0;
+    for (int i = 0; i < t.count; ++i) q += 4.0 * (double)cdiv(t.mats[i].s, 32) * (double)t.mats[i].l;
+    return q;
+  };
+  if (!eq_ids.empty()) {
+    // D init: column sums of squares of uX per 32-row block, then their sum
+    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.s, 256) * cdiv(d.l, kColStrip); },
+                  [&](const MatTable& t, int nb) {
+      ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t) + colsq_bytes(t), c.st);
+      return launch_colsq_partial(t, nb, c.st);
     }));
+    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
+      ProfScope ps(PC_AURORA, 0.0, colsq_bytes(t), c.st);
+      return launch_colsq_update(t, nb, 0, pe, beta, c.st);
+    }));
+  }
   const int rounds = eq_b.empty() ? 1 : c.cfg->pp_iterations;
   for (int k = 0; k < rounds; ++k) {
     if (!eq_ids.empty()) {
@@ -667,11 +704,20 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       for (int b : plain_b) { bids.push_back(b); in_q.push_back(false); fin.push_back(true); }
     muon_status s = stage_newton_schulz(c, bids, in_q, fin);
     if (s != MUON_OK) return s;
-    if (k < rounds - 1)
-      CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
+    if (k < rounds - 1) {
+      // D update: from the column sums the last update GEMM wrote (tensor-core
+      // mode), else from a pass over U
+      const bool tcq = c.cfg->gemm_mode == MUON_GEMM_BF16;
+      const auto fq = split_ids(c, eq_ids, [tcq](const MatDesc& d) { return tcq && d.colsq != nullptr; });
+      CK(for_chunks(c, fq.first, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
+        ProfScope ps(PC_AURORA, 0.0, colsq_bytes(t), c.st);
+        return launch_colsq_update(t, nb, 1, pe, beta, c.st);
+      }));
+      CK(for_chunks(c, fq.second, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
         return launch_colnorm(t, nb, 1, pe, beta, c.st);
       }));
+    }
   }
   return MUON_OK;
 }
@@ -812,6 +858,7 @@ const char* muon_status_string(muon_status s) {
     case MUON_ERR_WORKSPACE: return "workspace missing or too small";
     case MUON_ERR_CUDA: return "CUDA error";
     case MUON_ERR_TIMEOUT: return "device-side wait timed out";
+    case MUON_ERR_BOUNDS: return "index outside its buffer (checked build)";
   }
   return "unknown status";
 }
@@ -972,12 +1019,45 @@ muon_status muon_selftest_wait_timeout(long long max_cycles, void* stream) {
   return launch_wait_selftest(lim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
+// source line of the first failed index test seen by muon_last_device_status
+static unsigned int g_last_check_line = 0;
+
 muon_status muon_last_device_status(void* stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
   unsigned int v = 0, w = 0;
   if (read_and_clear_device_status(&v) != cudaSuccess) return MUON_ERR_CUDA;
   if (read_and_clear_gv_status(&w) != cudaSuccess) return MUON_ERR_CUDA;
-  return static_cast<muon_status>(v != 0 ? v : w);
+  unsigned int line = 0;
+  cudaError_t (*const readers[])(unsigned int*) = {read_and_clear_check_elementwise, read_and_clear_check_powiter,
+                                                   read_and_clear_check_gemm_tc, read_and_clear_check_gemm_simt,
+                                                   read_and_clear_check_adamw};
+  for (auto rd : readers) {
+    unsigned int q = 0;
+    if (rd(&q) != cudaSuccess) return MUON_ERR_CUDA;
+    if (q && !line) line = q;
+  }
+  if (line) g_last_check_line = line;
+  if (v != 0) return static_cast<muon_status>(v);
+  if (w != 0) return static_cast<muon_status>(w);
+  return line ? MUON_ERR_BOUNDS : MUON_OK;
+}
+
+int muon_build_checked(void) {
+#ifdef AURORA_MUON_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int muon_last_check_line(void) {
+  const unsigned int l = g_last_check_line;
+  g_last_check_line = 0;
+  return (int)l;
+}
+
+muon_status muon_selftest_bounds_check(void* stream) {
+  return launch_bounds_selftest(reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
 }  // extern "C"

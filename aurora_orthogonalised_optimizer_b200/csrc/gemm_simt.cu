@@ -7,6 +7,8 @@
 
 namespace am {
 
+AM_CHECK_READER(read_and_clear_check_gemm_simt)
+
 namespace {
 
 constexpr int BM = 64, BN = 64, BK = 16, NT = 256;
@@ -47,16 +49,19 @@ __global__ void __launch_bounds__(NT) k_gemm_simt(const GemmLaunch L) {
       {  // A tile: (m, k) at A[m * lda + k]
         const int mm = idx / BK, kk = idx % BK;
         const int gm = m0 + mm, gk = k0 + kk;
-        As[kk][mm] = (gm < g.M && gk < g.K) ? to_f(A[(int64_t)gm * g.lda + gk]) : 0.f;
+        As[kk][mm] = (gm < g.M && gk < g.K && AM_IN((int64_t)b * g.sa + (int64_t)gm * g.lda + gk, 1, (int64_t)g.count * g.sa))
+                         ? to_f(A[(int64_t)gm * g.lda + gk]) : 0.f;
       }
       if (b_nt) {  // (k, n) at B[n * ldb + k]
         const int nn = idx / BK, kk = idx % BK;
         const int gn = n0 + nn, gk = k0 + kk;
-        Bs[kk][nn] = (gn < g.N && gk < g.K) ? to_f(B[(int64_t)gn * g.ldb + gk]) : 0.f;
+        Bs[kk][nn] = (gn < g.N && gk < g.K && AM_IN((int64_t)b * g.sb + (int64_t)gn * g.ldb + gk, 1, (int64_t)g.count * g.sb))
+                         ? to_f(B[(int64_t)gn * g.ldb + gk]) : 0.f;
       } else {     // (k, n) at B[k * ldb + n]
         const int kk = idx / BN, nn = idx % BN;
         const int gn = n0 + nn, gk = k0 + kk;
-        Bs[kk][nn] = (gn < g.N && gk < g.K) ? to_f(B[(int64_t)gk * g.ldb + gn]) : 0.f;
+        Bs[kk][nn] = (gn < g.N && gk < g.K && AM_IN((int64_t)b * g.sb + (int64_t)gk * g.ldb + gn, 1, (int64_t)g.count * g.sb))
+                         ? to_f(B[(int64_t)gk * g.ldb + gn]) : 0.f;
       }
     }
     __syncthreads();
@@ -91,8 +96,10 @@ __global__ void __launch_bounds__(NT) k_gemm_simt(const GemmLaunch L) {
       const int gn = n0 + tx + 16 * j;
       if (gn >= g.N) continue;
       float v = alpha * acc[i][j];
-      if (E) v += beta * to_f(E[(int64_t)gm * g.lde + gn]);
-      C[(int64_t)gm * g.ldc + gn] = from_f<T>(v);
+      if (E && AM_IN((int64_t)b * g.se + (int64_t)gm * g.lde + gn, 1, (int64_t)g.count * g.se))
+        v += beta * to_f(E[(int64_t)gm * g.lde + gn]);
+      if (AM_IN((int64_t)b * g.sc + (int64_t)gm * g.ldc + gn, 1, (int64_t)g.count * g.sc))
+        C[(int64_t)gm * g.ldc + gn] = from_f<T>(v);
     }
   }
 }

@@ -41,6 +41,8 @@
 
 namespace am {
 
+AM_CHECK_READER(read_and_clear_check_gemm_tc)
+
 // Sticky per-device status word (a muon_status code; the first error wins).
 __device__ unsigned int g_device_status = 0;
 
@@ -145,6 +147,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y,
 }
 __device__ __forceinline__ void st_shared_u16(uint32_t a, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
 }
 __device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
   uint16_t v;
@@ -527,8 +534,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       uint4 en[4] = {}, un[4] = {};
       int next = 0;
       while (next < TBN / 32 && !wanted(next)) ++next;
-      if (next < TBN / 32 && Erow) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
-      if (next < TBN / 32 && Urow) load_e_chunk(Urow, ti.n0 + next * 32, G.N, un);
+      // element range of a 32-column chunk of this lane's row (for the checked build)
+      auto e_ok = [&](int64_t ld, int64_t stride, int col) {
+        return AM_IN((int64_t)ti.b * stride + (int64_t)row * ld + col, min(32, G.N - col), (int64_t)G.count * stride);
+      };
+      if (next < TBN / 32 && Erow && e_ok(G.lde, G.se, ti.n0 + next * 32)) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
+      if (next < TBN / 32 && Urow && e_ok(G.ldc, G.sc, ti.n0 + next * 32)) load_e_chunk(Urow, ti.n0 + next * 32, G.N, un);
       while (next < TBN / 32) {
         const int ch = next;
         const int col0 = ti.n0 + ch * 32;
@@ -536,8 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         const uint4 uc[4] = {un[0], un[1], un[2], un[3]};
         ++next;
         while (next < TBN / 32 && !wanted(next)) ++next;
-        if (next < TBN / 32 && Erow) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
-        if (next < TBN / 32 && Urow) load_e_chunk(Urow, ti.n0 + next * 32, G.N, un);
+        if (next < TBN / 32 && Erow && e_ok(G.lde, G.se, ti.n0 + next * 32)) load_e_chunk(Erow, ti.n0 + next * 32, G.N, en);
+        if (next < TBN / 32 && Urow && e_ok(G.ldc, G.sc, ti.n0 + next * 32)) load_e_chunk(Urow, ti.n0 + next * 32, G.N, un);
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TBN + ch * 32), r);
         uint32_t pk[16];
@@ -589,9 +600,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           for (int j = 0; j < 32; ++j)
             st_shared_u16(mbuf + swz64(j, 2 * lane), (uint16_t)(pk[j >> 1] >> (16 * (j & 1))));
         }
+        if (G.colsq) {
+          // column sums of the squared stored values of this 32 x 32 block:
+          // lane l sums columns 2 (l % 16), +1 over rows 16 (l / 16) .. +15
+          __syncwarp();
+          const int cp = lane & 15, rh = lane >> 4;
+          float q0 = 0.f, q1 = 0.f;
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const uint32_t w = ld_shared_u32(dbuf + swz64(16 * rh + r, 4 * cp));
+            const float v0 = bf16_bits_to_f(w & 0xFFFFu), v1 = bf16_bits_to_f(w >> 16);
+            q0 = fmaf(v0, v0, q0);
+            q1 = fmaf(v1, v1, q1);
+          }
+          q0 += __shfl_xor_sync(0xffffffffu, q0, 16);
+          q1 += __shfl_xor_sync(0xffffffffu, q1, 16);
+          const int64_t qo = (int64_t)ti.b * G.colsq_batch + (int64_t)(r0 >> 5) * G.colsq_ld + col0 + 2 * cp;
+          if (lane < 16 && AM_IN(qo, 2, (int64_t)G.count * G.colsq_batch))
+            *reinterpret_cast<float2*>(G.colsq + qo) = make_float2(q0, q1);
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0 && !G.no_store) {
           tma_store_3d(mC, dbuf, col0, r0, ti.b);
           if (mirror) tma_store_3d(mC, mbuf, r0, col0, ti.b);
           bulk_commit();
@@ -605,13 +635,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         s_cu = warp_sum(s_cu);
         if (lane == 0) {
           const int tin = ti.m0 / Gm::kTileM + G.tiles_m * (ti.n0 / TBN);
-          double* slot = G.dotp + ((int64_t)ti.b * G.tiles_per_mat + tin) * 16;
+          const int64_t so = ((int64_t)ti.b * G.tiles_per_mat + tin) * 16;
+          double* slot = G.dotp + so;
           const int w = (int)rank * 4 + q;
-          slot[2 * w] = (double)s_cc;
-          slot[2 * w + 1] = (double)s_cu;
-          if (!PAIR) {
-            slot[2 * (w + 4)] = 0.0;
-            slot[2 * (w + 4) + 1] = 0.0;
+          if (AM_IN(so, 16, (int64_t)G.count * G.tiles_per_mat * 16)) {
+            slot[2 * w] = (double)s_cc;
+            slot[2 * w + 1] = (double)s_cu;
+            if (!PAIR) {
+              slot[2 * (w + 4)] = 0.0;
+              slot[2 * (w + 4) + 1] = 0.0;
+            }
           }
         }
       }

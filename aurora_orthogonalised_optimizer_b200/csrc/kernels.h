@@ -37,6 +37,12 @@ struct GemmGroup {
   // dotp[((b * tiles_per_mat + tile) * 8 + warp) * 2 + {0, 1}].
   const void* dotu;
   double* dotp;
+  // Update kind, tensor-core path only: when colsq is set the epilogue also
+  // writes, per 32-row block of C, the column sums of the squared stored
+  // bf16 values: colsq[b * colsq_batch + (row / 32) * colsq_ld + col].
+  float* colsq;
+  int64_t colsq_ld, colsq_batch;
+  int no_store;                   // C itself is not needed (only colsq): skip its stores
 };
 
 constexpr int kMaxGemmGroups = 16;
@@ -83,6 +89,13 @@ cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int 
 cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, float beta,
                            cudaStream_t st);
 cudaError_t launch_scale_cols(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+// Aurora D from per-32-row-block column sums of squares (MatDesc::colsq):
+// k_colsq_partial forms them from uX (blocks of 256 rows x kColStrip columns);
+// the last update GEMM of a non-final polar forms them from U.
+// launch_colsq_update (one block per kColStrip columns) sums them:
+// mode 0 D init, mode 1 D update.
+cudaError_t launch_colsq_partial(const MatTable& t, int nblk, cudaStream_t st);
+cudaError_t launch_colsq_update(const MatTable& t, int nblk, int mode, float pp_eps, float beta, cudaStream_t st);
 cudaError_t launch_scalars(const MatTable& t, int op, int src_slot, float ns_eps, float contra,
                            float target_uw, double* scal, cudaStream_t st);
 cudaError_t launch_matvec(const MatTable& t, int nblk, int dir, cudaStream_t st);
@@ -122,5 +135,14 @@ cudaError_t launch_gramvec(const MatTable& t, int nblk, int mode, cudaStream_t s
 cudaError_t launch_gv_reduce(const MatTable& t, int normalise, cudaStream_t st);
 cudaError_t read_and_clear_gv_status(unsigned int* out);
 cudaError_t launch_sigma_out(const MatTable& t, const double* scal, float* sigma_out, cudaStream_t st);
+
+// Checked build: read and clear each file's check word (source line of the
+// first failed index test, 0 if none; always 0 in the normal build).
+cudaError_t read_and_clear_check_elementwise(unsigned int* out);
+cudaError_t read_and_clear_check_powiter(unsigned int* out);
+cudaError_t read_and_clear_check_gemm_tc(unsigned int* out);
+cudaError_t read_and_clear_check_gemm_simt(unsigned int* out);
+cudaError_t read_and_clear_check_adamw(unsigned int* out);
+cudaError_t launch_bounds_selftest(cudaStream_t st);
 
 }  // namespace am

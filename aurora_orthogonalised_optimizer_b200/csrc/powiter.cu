@@ -63,6 +63,8 @@ __device__ __forceinline__ uint32_t s_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 __device__ __forceinline__ void gv_raise(unsigned int code) { atomicCAS(&g_gv_status, 0u, code); }
+// elements of a matrix's per-item partials of X^T z (one ldl row per item)
+__device__ __forceinline__ int64_t gv_ext(const MatDesc& d) { return (d.s + d.gv_rows - 1) / d.gv_rows * d.ldl; }
 __device__ __forceinline__ void mb_init(uint32_t a, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
 }
@@ -253,6 +255,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
     // the group's rows are consecutive in X and in the stage: one copy (one
     // large bulk copy streams faster than one per row, and far faster than
     // smaller pieces)
+    if (!AM_IN(row0 * d.ldl, (int64_t)nrows * d.ldl, AM_EXT_X(d))) return;   // (the wait then times out)
     mb_expect_tx(fb, (uint32_t)nrows * row_bytes);
     bulk_g2s(ring + (uint32_t)s * kGvStageBytes, src + row0 * (int64_t)row_bytes, (uint32_t)nrows * row_bytes, fb);
   };
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
     coff[k] = (uint32_t)c * Tr::kChunkBytes;
     cval[k] = (k < KC && c < C) ? (int)min((int64_t)8, d.l - j) : 0;
     float yy[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (mode != GV_ACC && cval[k] == 8) {
+    if (mode != GV_ACC && cval[k] == 8 && AM_IN(j, 8, AM_EXT_VEC(d))) {
       const float4 a = reinterpret_cast<const float4*>(yv + j)[0];
       const float4 b = reinterpret_cast<const float4*>(yv + j)[1];
       yy[0] = a.x; yy[1] = a.y; yy[2] = a.z; yy[3] = a.w;
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
     } else if (mode != GV_ACC) {
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        if (e < cval[k]) yy[e] = yv[j + e];
+        if (e < cval[k] && AM_IN(j + e, 1, AM_EXT_VEC(d))) yy[e] = yv[j + e];
     }
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
     float z[RM];
     if (mode == GV_ACC) {
 #pragma unroll
-      for (int r = 0; r < RM; ++r) z[r] = r < nr ? zv[i0 + r] : 0.f;
+      for (int r = 0; r < RM; ++r) z[r] = r < nr && AM_IN(i0 + r, 1, AM_EXT_VEC(d)) ? zv[i0 + r] : 0.f;
     } else {
       unsigned long long p2[RM];
 #pragma unroll
@@ -374,7 +377,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
       if (tt == 0)
 #pragma unroll
         for (int r = 0; r < RM; ++r)
-          if (r < nr) zv[i0 + r] = z[r];
+          if (r < nr && AM_IN(i0 + r, 1, AM_EXT_VEC(d))) zv[i0 + r] = z[r];
     }
     if (mode != GV_DOT) {
 #pragma unroll
@@ -407,8 +410,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
     if (cval[k] > 0) {
       const float2 a0 = upk2(acc2[k][0]), a1 = upk2(acc2[k][1]), a2 = upk2(acc2[k][2]), a3 = upk2(acc2[k][3]);
       float4* q = reinterpret_cast<float4*>(dst + 8 * (int64_t)(tt + k * 32 * TW));
-      q[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
-      q[1] = make_float4(a2.x, a2.y, a3.x, a3.y);
+      if (NT == 1 ? AM_IN((int64_t)item * d.ldl + 8 * (int64_t)(tt + k * 32 * TW), 8, gv_ext(d))
+                  : AM_IN((int64_t)team * d.ldl + 8 * (int64_t)(tt + k * 32 * TW), 8, (int64_t)NT * d.ldl)) {
+        q[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
+        q[1] = make_float4(a2.x, a2.y, a3.x, a3.y);
+      }
     }
   }
   if (NT == 1) return;
@@ -421,7 +427,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gramvec(const MatTable t, int
       const float4 v = reinterpret_cast<const float4*>(comb + (int64_t)tm * d.ldl)[j4];
       sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
     }
-    reinterpret_cast<float4*>(part)[j4] = sum;
+    if (AM_IN((int64_t)item * d.ldl + 4 * (int64_t)j4, 4, gv_ext(d))) reinterpret_cast<float4*>(part)[j4] = sum;
   }
 }
 
@@ -441,6 +447,7 @@ __global__ void __launch_bounds__(512) k_gv_reduce(const MatTable t, int normali
     const float* p = d.gvp + 8 * (int64_t)c;
 #pragma unroll 6
     for (int q = 0; q < P; ++q) {   // item order: the sum is the same on every run
+      if (!AM_IN((int64_t)q * d.ldl + 8 * (int64_t)c, 8, gv_ext(d))) continue;
       const float4 a = __ldg(reinterpret_cast<const float4*>(p + (int64_t)q * d.ldl));
       const float4 b = __ldg(reinterpret_cast<const float4*>(p + (int64_t)q * d.ldl) + 1);
       v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
@@ -449,7 +456,7 @@ __global__ void __launch_bounds__(512) k_gv_reduce(const MatTable t, int normali
     const int64_t j = 8 * (int64_t)c;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if (j + e < d.l) {
+      if (j + e < d.l && AM_IN(j + e, 1, AM_EXT_VEC(d))) {
         out[j + e] = v[e];
         ss += (double)v[e] * v[e];
       }
@@ -458,7 +465,8 @@ __global__ void __launch_bounds__(512) k_gv_reduce(const MatTable t, int normali
   if (!normalise) return;
   if (d.tall) {
     ss = 0.0;
-    for (int64_t i = threadIdx.x; i < d.s; i += blockDim.x) ss += (double)d.vec0[i] * d.vec0[i];
+    for (int64_t i = threadIdx.x; i < d.s; i += blockDim.x)
+      if (AM_IN(i, 1, AM_EXT_VEC(d))) ss += (double)d.vec0[i] * d.vec0[i];
   }
   ss = block_sum(ss, red);
   const float inv = (float)(1.0 / fmax(sqrt(ss), 1e-30));
@@ -466,7 +474,7 @@ __global__ void __launch_bounds__(512) k_gv_reduce(const MatTable t, int normali
     const int64_t j = 8 * (int64_t)c;
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      if (j + e < d.l) out[j + e] *= inv;
+      if (j + e < d.l && AM_IN(j + e, 1, AM_EXT_VEC(d))) out[j + e] *= inv;
   }
 }
 
@@ -509,6 +517,8 @@ cudaError_t launch_gv_reduce(const MatTable& t, int normalise, cudaStream_t st) 
   k_gv_reduce<<<t.count, 512, 0, st>>>(t, normalise);
   return cudaGetLastError();
 }
+
+AM_CHECK_READER(read_and_clear_check_powiter)
 
 cudaError_t read_and_clear_gv_status(unsigned int* out) {
   unsigned int v = 0, zero = 0;

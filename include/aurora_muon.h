@@ -44,7 +44,9 @@ typedef enum {
   MUON_ERR_UNSUPPORTED = 2,  /* a valid request the library does not implement */
   MUON_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than muon_workspace_size() */
   MUON_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
-  MUON_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up (see muon_last_device_status) */
+  MUON_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up (see muon_last_device_status) */
+  MUON_ERR_BOUNDS = 6        /* checked build only: a kernel's index fell outside its buffer
+                                (the access was skipped; see muon_build_checked) */
 } muon_status;
 
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
@@ -211,9 +213,26 @@ muon_status adamw_step(const adamw_config* cfg, int n, const int64_t* numels, co
                        float* const* exp_avg_sq, void* stream);
 
 /* Synchronises `stream`, then returns and clears the sticky device status
- * word of the current device (MUON_OK, or MUON_ERR_TIMEOUT after a bounded
- * device wait gave up). */
+ * words of the current device: MUON_OK, MUON_ERR_TIMEOUT after a bounded
+ * device wait gave up, or (checked build) MUON_ERR_BOUNDS after an index
+ * check failed. */
 muon_status muon_last_device_status(void* stream);
+
+/* Debugging aid without a counterpart on the pages (the pool has no memory
+ * sanitizer).  libaurora_muon_checked.so is the same library compiled with
+ * every global access of the streaming, power-iteration and GEMM-epilogue
+ * kernels tested against the extent of the buffer it addresses (TMA loads
+ * and stores are bounded by their tensor maps); a failed test skips the
+ * access and records MUON_ERR_BOUNDS.  muon_build_checked() returns 1 in
+ * that library and 0 in libaurora_muon.so.  muon_last_check_line() returns
+ * (and clears) the source line of the first failed test, 0 if none.
+ * muon_selftest_bounds_check launches one thread that tests an element
+ * range lying outside a 4-element extent without touching memory: in the
+ * checked library the next muon_last_device_status returns MUON_ERR_BOUNDS,
+ * in the normal one MUON_OK. */
+int muon_build_checked(void);
+int muon_last_check_line(void);
+muon_status muon_selftest_bounds_check(void* stream);
 
 /* Diagnostic of the failure-detection path (no counterpart on the pages):
  * launches one block whose thread waits, with the same bounded-wait routine

@@ -26,3 +26,14 @@ def lib():
     """The C-ABI library (loads on CPU; compute calls need a GPU)."""
     from aurora_orthogonalised_optimizer_b200 import _abi
     return _abi.load()
+
+
+@pytest.fixture(autouse=True)
+def _checked_build_status(request):
+    """Under the bounds-checked library (AURORA_MUON_CHECKED=1) every GPU test
+    must also leave no failed index test behind."""
+    yield
+    if os.environ.get("AURORA_MUON_CHECKED") == "1" and request.node.get_closest_marker("gpu"):
+        from aurora_orthogonalised_optimizer_b200 import _abi as A
+        st = A.last_device_status()
+        assert st == A.MUON_OK, (A.status_string(st), "line", A.last_check_line())

@@ -178,3 +178,20 @@ def test_noalloc_entry_rejects_oversized_edges_on_the_host(lib):
     code = lib.opnorm_normalize_noalloc(C.byref(cfg.to_c()), 1, A._shapes([(1 << 31, 1 << 31)]), ptrs,
                                         A.MUON_F32, None, None, None)
     assert code == A.MUON_ERR_UNSUPPORTED          # inside the edge bound, beyond the scratch
+
+
+def test_checked_library_exports_the_same_symbols():
+    """The bounds-checked build (libaurora_muon_checked.so) loads on the host,
+    exports every declared symbol and says it is the checked one."""
+    path = A.CHECKED_LIB_PATH
+    assert os.path.exists(path), "build it with build.py --checked"
+    chk = C.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(chk, name), name
+    chk.muon_build_checked.restype = C.c_int
+    assert chk.muon_build_checked() == 1
+    plain = C.CDLL(A.LIB_PATH)
+    plain.muon_build_checked.restype = C.c_int
+    assert plain.muon_build_checked() == 0
+    chk.muon_status_string.restype = C.c_char_p
+    assert b"checked build" in chk.muon_status_string(A.MUON_ERR_BOUNDS)
