@@ -182,23 +182,24 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
   }
 }
 
-// Column sums of squares of uX over 32-row blocks, into MatDesc::colsq
-// ([ceil(s / 32)][round64(l)] floats): a block covers 256 rows x 256 columns,
-// warp w rows 32 w .. +31 of them, each lane 8 columns (one 16-byte load per
-// row).  Many short independent blocks instead of one block walking every
-// row of a column strip.
-__global__ void __launch_bounds__(kEwThreads)
+// Column sums of squares of uX over kColsqRows-row blocks, into
+// MatDesc::colsq ([ceil(s / kColsqRows)][round64(l)] floats): a block covers
+// 8 kColsqRows rows x 256 columns, warp w rows kColsqRows w .. of them, each
+// lane 8 columns (one 16-byte load per row).  Blocks of bounded length
+// instead of one block walking every row of a column strip (whose last wave
+// leaves most of the GPU idle).
+__global__ void __launch_bounds__(kEwThreads, 4)
 k_colsq_partial(const MatTable t) {
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int64_t strips = (d.l + kColStrip - 1) / kColStrip;
   const int64_t b = blockIdx.x - t.blk_prefix[mi];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t rb = (b / strips) * 8 + w;                  // 32-row block of this warp
+  const int64_t rb = (b / strips) * 8 + w;                  // row block of this warp
   const int64_t j = (b % strips) * kColStrip + 8 * lane;
-  const int64_t i0 = rb * 32;
+  const int64_t i0 = rb * kColsqRows;
   if (i0 >= d.s || j >= d.l) return;
-  const int64_t i1 = min(d.s, i0 + 32);
+  const int64_t i1 = min(d.s, i0 + kColsqRows);
   const bool vec = (d.ldl & 7) == 0;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
@@ -210,23 +211,24 @@ k_colsq_partial(const MatTable t) {
   }
   float* q = d.colsq + rb * ((d.l + 63) / 64 * 64) + j;     // j + 8 <= round64(l)
   if (!AM_IN(rb * ((d.l + 63) / 64 * 64) + j, 8, ((d.s + 31) / 32) * ((d.l + 63) / 64 * 64))) return;
+  // (ceil(s / kColsqRows) row blocks fit the buffer sized for 32-row blocks)
   reinterpret_cast<float4*>(q)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
   reinterpret_cast<float4*>(q)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
 // Aurora D from the partial column sums in MatDesc::colsq (written per
-// 32-row block by k_colsq_partial from uX, or by the last update GEMM of the
-// previous polar from U): one thread per column sums the ceil(s / 32)
-// partials in block order (deterministic).
+// kColsqRows-row block by k_colsq_partial from uX, or per 32-row block by the
+// last update GEMM of the previous polar from U): one thread per column sums
+// the ceil(s / rows) partials in block order (deterministic).
 //   mode 0 (D init):  D_j = 1 / max(sqrt(sum), pp_eps)
 //   mode 1 (D update): D_j *= (target / max(sum, pp_eps^2))^beta, target = s / l
 __global__ void __launch_bounds__(kColStrip)
-k_colsq_update(const MatTable t, int mode, float pp_eps, float beta) {
+k_colsq_update(const MatTable t, int mode, int rows, float pp_eps, float beta) {
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int64_t j = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kColStrip + threadIdx.x;
   if (j >= d.l) return;
-  const int64_t nb = (d.s + 31) / 32, ldq = (d.l + 63) / 64 * 64;
+  const int64_t nb = (d.s + rows - 1) / rows, ldq = (d.l + 63) / 64 * 64;
   const float* q = d.colsq + j;
   float sum = 0.f;
   for (int64_t b = 0; b < nb; ++b)
@@ -796,6 +798,47 @@ k_scale_cols_flat_bf16(const MatTable t, double* partials) {
   }
 }
 
+// bf16 Newton-Schulz storage, rows contiguous: X0 = uX diag(D) by column
+// strips.  A block owns kStripCols columns (8 per thread) over kStripRows
+// rows; each thread loads its 8 column scales once and walks its columns down
+// the rows, four rows' loads in flight, one 16-byte load and one store per
+// row (the chunk-wise kernel above re-reads the scales for every 8 elements).
+// Partial |X0|^2 per warp, one slot per block.
+__global__ void __launch_bounds__(kEwThreads, 4)
+k_scale_cols_strip_bf16(const MatTable t, double* partials) {
+  const int mi = find_mat(t, blockIdx.x);
+  const MatDesc& d = t.mats[mi];
+  const int64_t strips = (d.l + kStripCols - 1) / kStripCols;
+  const int64_t b = blockIdx.x - t.blk_prefix[mi];
+  const int64_t j = (b % strips) * kStripCols + 8 * threadIdx.x;
+  const int64_t i0 = (b / strips) * kStripRows, i1 = min(d.s, i0 + kStripRows);
+  const __nv_bfloat16* uX = reinterpret_cast<const __nv_bfloat16*>(d.uX);
+  float s2 = 0.f;
+  if (j < d.l) {                                     // l is a multiple of 8: the whole group is inside
+    float dd[8];
+    ld8c(d.l, d.D, j, kF32, dd);
+    for (int64_t i = i0; i < i1; i += 4) {
+      uint4 x[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        x[r] = i + r < i1 ? LDG8BF(AM_EXT_X(d), uX, (i + r) * d.ldl + j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (i + r >= i1) break;
+        float v[8];
+        bf16x8_to_f32(x[r], v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          v[q] *= dd[q];
+          s2 += v[q] * v[q];
+        }
+        st8c(AM_EXT_X(d), d.X0, (i + r) * d.ldl + j, kBF16, v);
+      }
+    }
+  }
+  if (AM_IN(b, 1, d.nslots)) warp_partials(partials, d.part + b, 1, s2, 0.f);
+}
+
 __global__ void __launch_bounds__(kEwThreads)
 k_dots_flat(const MatTable t, double* partials) {
   const int mi = find_mat(t, blockIdx.x);
@@ -1134,7 +1177,7 @@ cudaError_t launch_colsq_partial(const MatTable& t, int nblk, cudaStream_t st) {
 }
 cudaError_t launch_colsq_update(const MatTable& t, int nblk, int mode, float pp_eps, float beta, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
-  k_colsq_update<<<nblk, kColStrip, 0, st>>>(t, mode, pp_eps, beta);
+  k_colsq_update<<<nblk, kColStrip, 0, st>>>(t, mode, mode == 0 ? kColsqRows : 32, pp_eps, beta);
   return cudaGetLastError();
 }
 cudaError_t launch_scale_cols(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
@@ -1174,6 +1217,11 @@ cudaError_t launch_prologue_tall_bf16(const MatTable& t, int nblk, float mu, int
                                       double* partials, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   k_prologue_tall_bf16<<<nblk, kEwThreads, 0, st>>>(t, mu, nesterov, want_w2, partials);
+  return cudaGetLastError();
+}
+cudaError_t launch_scale_cols_strip_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
+  if (nblk == 0) return cudaSuccess;
+  k_scale_cols_strip_bf16<<<nblk, kEwThreads, 0, st>>>(t, partials);
   return cudaGetLastError();
 }
 cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st) {

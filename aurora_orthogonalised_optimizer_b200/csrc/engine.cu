@@ -659,37 +659,45 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       if (e != cudaSuccess) return e;
       return launch_copy_rho(t, c.scal, c.st);
     }));
-  auto colsq_bytes = [](const MatTable& t) {
+  // bytes of the column-sum partials (one float per column per row block)
+  auto colsq_bytes = [](const MatTable& t, int rows) {
     double q = 0.0;
-    for (int i = 0; i < t.count; ++i) q += 4.0 * (double)cdiv(t.mats[i].s, 32) * (double)t.mats[i].l;
+    for (int i = 0; i < t.count; ++i) q += 4.0 * (double)cdiv(t.mats[i].s, rows) * (double)t.mats[i].l;
     return q;
   };
   if (!eq_ids.empty()) {
     // D init: column sums of squares of uX per 32-row block, then their sum
-    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.s, 256) * cdiv(d.l, kColStrip); },
+    CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.s, 8 * kColsqRows) * cdiv(d.l, kColStrip); },
                   [&](const MatTable& t, int nb) {
-      ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t) + colsq_bytes(t), c.st);
+      ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t) + colsq_bytes(t, kColsqRows), c.st);
       return launch_colsq_partial(t, nb, c.st);
     }));
     CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
-      ProfScope ps(PC_AURORA, 0.0, colsq_bytes(t), c.st);
+      ProfScope ps(PC_AURORA, 0.0, colsq_bytes(t, kColsqRows), c.st);
       return launch_colsq_update(t, nb, 0, pe, beta, c.st);
     }));
   }
   const int rounds = eq_b.empty() ? 1 : c.cfg->pp_iterations;
   for (int k = 0; k < rounds; ++k) {
     if (!eq_ids.empty()) {
+      // bf16 storage with contiguous rows: by column strips; else flat chunks
+      // or 64 x 64 tiles.  The partial slots each form leaves differ, and the
+      // sum below reads exactly those.
+      const bool bf16 = c.plan->ns_dtype == kBF16;
+      auto strip_blocks = [](const MatDesc& d) { return cdiv(d.l, kStripCols) * cdiv(d.s, kStripRows); };
       const auto fx = split_ids(c, eq_ids, flat_x);
-      CK(for_chunks(c, fx.first, fblocks_x, [&](const MatTable& t, int nb) {
+      CK(for_chunks(c, fx.first, [&](const MatDesc& d) { return bf16 ? strip_blocks(d) : fblocks_x(d); },
+                    [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
-        return c.plan->ns_dtype == kBF16 ? launch_scale_cols_flat_bf16(t, nb, c.partials, c.st)
-                                         : launch_scale_cols_flat(t, nb, c.partials, c.st);
+        return bf16 ? launch_scale_cols_strip_bf16(t, nb, c.partials, c.st)
+                    : launch_scale_cols_flat(t, nb, c.partials, c.st);
       }));
       CK(for_chunks(c, fx.second, blocks_x, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, 2.0 * c.plan->nsb * table_elems(t), c.st);
         return launch_scale_cols(t, nb, c.partials, c.st);
       }));
-      CK(for_chunks(c, eq_ids, slots_x, [&](const MatTable& t, int) {
+      CK(for_chunks(c, eq_ids, [&](const MatDesc& d) { return bf16 && flat_x(d) ? strip_blocks(d) : slots_x(d); },
+                    [&](const MatTable& t, int) {
         ProfScope ps(PC_REDUCE, 0.0, 0.0, c.st);
         cudaError_t e = launch_finalize_sums(t, c.partials, 1, S_SUM_X02, -1, c.scal, c.st);
         if (e != cudaSuccess) return e;
@@ -710,7 +718,7 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       const bool tcq = c.cfg->gemm_mode == MUON_GEMM_BF16;
       const auto fq = split_ids(c, eq_ids, [tcq](const MatDesc& d) { return tcq && d.colsq != nullptr; });
       CK(for_chunks(c, fq.first, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
-        ProfScope ps(PC_AURORA, 0.0, colsq_bytes(t), c.st);
+        ProfScope ps(PC_AURORA, 0.0, colsq_bytes(t, 32), c.st);
         return launch_colsq_update(t, nb, 1, pe, beta, c.st);
       }));
       CK(for_chunks(c, fq.second, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {

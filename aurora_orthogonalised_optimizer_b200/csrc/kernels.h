@@ -89,11 +89,13 @@ cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int 
 cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, float beta,
                            cudaStream_t st);
 cudaError_t launch_scale_cols(const MatTable& t, int nblk, double* partials, cudaStream_t st);
-// Aurora D from per-32-row-block column sums of squares (MatDesc::colsq):
-// k_colsq_partial forms them from uX (blocks of 256 rows x kColStrip columns);
-// the last update GEMM of a non-final polar forms them from U.
-// launch_colsq_update (one block per kColStrip columns) sums them:
-// mode 0 D init, mode 1 D update.
+// Aurora D from per-row-block column sums of squares (MatDesc::colsq):
+// k_colsq_partial forms them from uX per kColsqRows rows (blocks of
+// 8 kColsqRows rows x kColStrip columns); the last update GEMM of a
+// non-final polar forms them from U per 32 rows.  launch_colsq_update (one
+// block per kColStrip columns) sums them: mode 0 D init (kColsqRows-row
+// partials), mode 1 D update (32-row partials).
+constexpr int kColsqRows = 128;
 cudaError_t launch_colsq_partial(const MatTable& t, int nblk, cudaStream_t st);
 cudaError_t launch_colsq_update(const MatTable& t, int nblk, int mode, float pp_eps, float beta, cudaStream_t st);
 cudaError_t launch_scalars(const MatTable& t, int op, int src_slot, float ns_eps, float contra,
@@ -109,6 +111,11 @@ cudaError_t launch_prologue_tall_bf16(const MatTable& t, int nblk, float mu, int
                                       double* partials, cudaStream_t st);
 // Flat Aurora input scaling with bf16 NS storage.
 cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st);
+// The same by column strips: blocks of kStripCols columns x kStripRows rows,
+// one partial slot per block (cdiv(l, kStripCols) * cdiv(s, kStripRows) of
+// them, never more than the matrix's 64 x 64 tiles).
+constexpr int kStripCols = 2048, kStripRows = 64;
+cudaError_t launch_scale_cols_strip_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st);
 // Flat (wide / square, rows a multiple of 8) and bf16 params and NS storage.
 cudaError_t launch_epilogue_flat_bf16(const MatTable& t, int nblk, float lr, int update_w, const double* scal,
                                       cudaStream_t st);
