@@ -324,7 +324,7 @@ def build_checked() -> bool:
 
 
 def last_check_line() -> int:
-    """Source line of the first failed index test (checked build), 0 if none."""
+    """Where the first failed index test sits (checked build): file * 100000 + line, 0 if none."""
     return int(load().muon_last_check_line())
 
 

@@ -82,10 +82,11 @@ __device__ __forceinline__ void st8r(void* p, int64_t row_off, int64_t j, int64_
 
 // ---------------------------------------------------------------- checked build
 // Built with AURORA_MUON_CHECKED (build.py --checked -> libaurora_muon_checked.so),
-// every global access of the streaming, power-iteration and GEMM-epilogue
-// kernels first tests its element range [first, first + count) against the
-// extent of the buffer it addresses.  A failed test records the source line
-// in this file's sticky check word (first failure wins) and the access is
+// every global access of the streaming, power-iteration, GEMM-epilogue,
+// SIMT-GEMM and AdamW kernels first tests its element range
+// [first, first + count) against the extent of the buffer it addresses (TMA
+// loads and stores are bounded by their tensor maps).  A failed test records
+// the source line in the file's sticky check word (first failure wins) and the access is
 // skipped (loads read zeros), so nothing outside a buffer is touched; the
 // host reads the words through muon_last_device_status (MUON_ERR_BOUNDS).
 // In the normal build the test is the constant true and compiles away.
@@ -195,8 +196,9 @@ struct MatDesc {
   float* vec1;
   float* rho_slot;    // bucket-ordered copy of rho read by the GEMM epilogues
   float* gvp;         // fused power iteration: one partial X^T z (ldl floats) per row item
-  float* colsq;       // Aurora D update: column sums of U^2 (X orientation) per 32-row block,
-                      // [ceil(s / 32)][round64(l)] floats, written by the last update GEMM
+  float* colsq;       // Aurora D: column sums of squares (X orientation) per row block, room for
+                      // [ceil(s / 32)][round64(l)] floats: of uX per 128 rows for the D init,
+                      // of U per 32 rows (written by the last update GEMM) for the D update
   int64_t m, n, s, l, ldl;
   int tall;           // m > n
   int idx;            // matrix index (scalar block row)

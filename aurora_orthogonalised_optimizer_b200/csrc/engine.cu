@@ -133,11 +133,10 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
     b.off_dots = off;
     off = align_up(off + b.members.size() * (size_t)b.dot_tiles * 16 * sizeof(double));
   }
-  // column sums of U^2 for Aurora's D update, written by the last update GEMM
-  // of each non-final polar (tensor-core mode, non-square buckets)
-  // column sums of squares per 32-row block for Aurora's D (non-square
-  // buckets): formed from uX for the D init; for the D updates, written by
-  // the last update GEMM of each non-final polar in the tensor-core mode
+  // column sums of squares per row block for Aurora's D (non-square
+  // buckets), sized for 32-row blocks: formed from uX for the D init; for the
+  // D updates, written by the last update GEMM of each non-final polar in the
+  // tensor-core mode
   for (auto& b : p.buckets) {
     b.colsq = cfg->aurora && b.s != b.l;
     b.colsq_gemm = b.colsq && cfg->gemm_mode == MUON_GEMM_BF16 && cfg->pp_iterations > 1;
@@ -666,7 +665,7 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
     return q;
   };
   if (!eq_ids.empty()) {
-    // D init: column sums of squares of uX per 32-row block, then their sum
+    // D init: column sums of squares of uX per kColsqRows-row block, then their sum
     CK(for_chunks(c, eq_ids, [](const MatDesc& d) { return cdiv(d.s, 8 * kColsqRows) * cdiv(d.l, kColStrip); },
                   [&](const MatTable& t, int nb) {
       ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t) + colsq_bytes(t, kColsqRows), c.st);
@@ -1027,7 +1026,7 @@ muon_status muon_selftest_wait_timeout(long long max_cycles, void* stream) {
   return launch_wait_selftest(lim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
-// source line of the first failed index test seen by muon_last_device_status
+// the first failed index test seen by muon_last_device_status (file * 100000 + line)
 static unsigned int g_last_check_line = 0;
 
 muon_status muon_last_device_status(void* stream) {
@@ -1035,14 +1034,15 @@ muon_status muon_last_device_status(void* stream) {
   unsigned int v = 0, w = 0;
   if (read_and_clear_device_status(&v) != cudaSuccess) return MUON_ERR_CUDA;
   if (read_and_clear_gv_status(&w) != cudaSuccess) return MUON_ERR_CUDA;
+  // the first failed index test, as file * 100000 + line (files in this order, from 1)
   unsigned int line = 0;
   cudaError_t (*const readers[])(unsigned int*) = {read_and_clear_check_elementwise, read_and_clear_check_powiter,
                                                    read_and_clear_check_gemm_tc, read_and_clear_check_gemm_simt,
                                                    read_and_clear_check_adamw};
-  for (auto rd : readers) {
+  for (unsigned int f = 0; f < 5; ++f) {
     unsigned int q = 0;
-    if (rd(&q) != cudaSuccess) return MUON_ERR_CUDA;
-    if (q && !line) line = q;
+    if (readers[f](&q) != cudaSuccess) return MUON_ERR_CUDA;
+    if (q && !line) line = (f + 1) * 100000u + q;
   }
   if (line) g_last_check_line = line;
   if (v != 0) return static_cast<muon_status>(v);

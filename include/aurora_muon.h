@@ -225,7 +225,9 @@ muon_status muon_last_device_status(void* stream);
  * and stores are bounded by their tensor maps); a failed test skips the
  * access and records MUON_ERR_BOUNDS.  muon_build_checked() returns 1 in
  * that library and 0 in libaurora_muon.so.  muon_last_check_line() returns
- * (and clears) the source line of the first failed test, 0 if none.
+ * (and clears) where the first failed test sits, 0 if none: file * 100000 +
+ * line, files numbered 1 elementwise.cu, 2 powiter.cu, 3 gemm_tc.cu,
+ * 4 gemm_simt.cu, 5 adamw.cu.
  * muon_selftest_bounds_check launches one thread that tests an element
  * range lying outside a 4-element extent without touching memory: in the
  * checked library the next muon_last_device_status returns MUON_ERR_BOUNDS,
