@@ -135,23 +135,23 @@ __global__ void k_finalize_sums(const MatTable t, const double* partials, int nq
 }
 
 // ============================================================================
-// Column reductions over the X orientation (s x l): per column j of X
-// (= a row of the tall-oriented matrix), sum_i X_ij^2.
-//   mode 0 (D init):  D_j = 1 / max(sqrt(sum), pp_eps)              ["源码实现"]
-//   mode 1 (D update): row_sq = max(sum, pp_eps^2);
-//                      D_j *= (target / row_sq)^beta, target = s / l
+// Aurora D update from a pass over U (the FP32 / SIMT modes; the tensor-core
+// mode takes the column sums from the GEMM epilogue): per column j of the X
+// orientation (= a row of the tall-oriented matrix) sum_i U_ij^2, then
+// row_sq = max(sum, pp_eps^2) and D_j *= (target / row_sq)^beta with
+// target = s / l ["源码实现"].
 // A block owns kColStrip = 256 columns; each warp streams every 8th row with
 // one 16-byte load (8 columns) per lane, so a warp reads 512 contiguous bytes.
 // ============================================================================
 __global__ void __launch_bounds__(kEwThreads)
-k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
+k_colnorm(const MatTable t, float pp_eps, float beta) {
   __shared__ float part[kWarps][kColStrip];
   const int mi = find_mat(t, blockIdx.x);
   const MatDesc& d = t.mats[mi];
   const int b = blockIdx.x - t.blk_prefix[mi];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t j = (int64_t)b * kColStrip + 8 * lane;
-  const void* X = mode == 0 ? d.uX : d.UX;
+  const void* X = d.UX;
   const bool vec = (d.ldl & 7) == 0;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (j < d.l) {
@@ -172,13 +172,9 @@ k_colnorm(const MatTable t, int mode, float pp_eps, float beta) {
 #pragma unroll
     for (int r = 0; r < kWarps; ++r) sum += part[r][threadIdx.x];
     if (!AM_IN(jj, 1, d.l)) return;
-    if (mode == 0) {
-      d.D[jj] = 1.f / fmaxf(sqrtf(sum), pp_eps);
-    } else {
-      const float row_sq = fmaxf(sum, pp_eps * pp_eps);
-      const float target = (float)d.s / (float)d.l;
-      d.D[jj] = d.D[jj] * powf(target / row_sq, beta);
-    }
+    const float row_sq = fmaxf(sum, pp_eps * pp_eps);
+    const float target = (float)d.s / (float)d.l;
+    d.D[jj] = d.D[jj] * powf(target / row_sq, beta);
   }
 }
 
@@ -729,80 +725,12 @@ k_scale_cols_flat(const MatTable t, double* partials) {
   }
 }
 
-// bf16 Newton-Schulz storage: the same scaling with each chunk's loads (u
-// and the column scales) issued while the previous chunk is processed.
-__global__ void __launch_bounds__(kEwThreads)
-k_scale_cols_flat_bf16(const MatTable t, double* partials) {
-  const int mi = find_mat(t, blockIdx.x);
-  const MatDesc& d = t.mats[mi];
-  const int64_t total = d.s * d.l;
-  const int64_t c0 = (int64_t)(blockIdx.x - t.blk_prefix[mi]) * kEwTilesPerCta;
-  const int64_t c1 = min(c0 + kEwTilesPerCta, (total + kFlatChunk - 1) / kFlatChunk);
-  const __nv_bfloat16* uX = reinterpret_cast<const __nv_bfloat16*>(d.uX);
-  auto off = [&](int64_t c, int k) { return c * kFlatChunk + 8 * (threadIdx.x + kEwThreads * k); };
-  // column of each of this thread's two 8-groups in the chunk load() fetches
-  // next: chunks are loaded in order, so it advances by kFlatChunk mod l
-  // (one division per block instead of one per group)
-  const int64_t step = kFlatChunk % d.l;
-  int64_t col[2] = {off(c0, 0) % d.l, off(c0, 1) % d.l};
-  auto load = [&](int64_t c, uint4 (&x)[2], float4 (&dj)[2][2]) {
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t e = off(c, k);
-      if (e < total) {
-        x[k] = LDG8BF(AM_EXT_X(d), uX, e);
-        const float4* dp = reinterpret_cast<const float4*>(d.D + col[k]);
-        if (AM_IN(col[k], 8, d.l)) {
-          dj[k][0] = __ldg(dp);
-          dj[k][1] = __ldg(dp + 1);
-        } else {
-          dj[k][0] = dj[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      } else {
-        x[k] = make_uint4(0, 0, 0, 0);
-        dj[k][0] = dj[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      col[k] += step;
-      if (col[k] >= d.l) col[k] -= d.l;
-    }
-  };
-  auto process = [&](int64_t c, const uint4 (&x)[2], const float4 (&dj)[2][2]) {
-    float s2 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t e = off(c, k);
-      if (e >= total) continue;
-      float v[8];
-      bf16x8_to_f32(x[k], v);
-      const float dd[8] = {dj[k][0].x, dj[k][0].y, dj[k][0].z, dj[k][0].w,
-                           dj[k][1].x, dj[k][1].y, dj[k][1].z, dj[k][1].w};
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        v[q] *= dd[q];
-        s2 += v[q] * v[q];
-      }
-      st8c(AM_EXT_X(d), d.X0, e, kBF16, v);
-    }
-    if (AM_IN(c, 1, d.nslots)) warp_partials(partials, d.part + c, 1, s2, 0.f);
-  };
-  if (c0 >= c1) return;
-  uint4 xa[2], xb[2];
-  float4 da[2][2], db[2][2];
-  load(c0, xa, da);
-  for (int64_t c = c0; c < c1; c += 2) {
-    if (c + 1 < c1) load(c + 1, xb, db);
-    process(c, xa, da);
-    if (c + 1 >= c1) break;
-    if (c + 2 < c1) load(c + 2, xa, da);
-    process(c + 1, xb, db);
-  }
-}
-
 // bf16 Newton-Schulz storage, rows contiguous: X0 = uX diag(D) by column
 // strips.  A block owns kStripCols columns (8 per thread) over kStripRows
 // rows; each thread loads its 8 column scales once and walks its columns down
 // the rows, four rows' loads in flight, one 16-byte load and one store per
-// row (the chunk-wise kernel above re-reads the scales for every 8 elements).
+// row (the chunk-wise kernel above re-reads the scales for every 8 elements;
+// its bf16 form ran at 77% of HBM against this one's 100% under ncu).
 // Partial |X0|^2 per warp, one slot per block.
 __global__ void __launch_bounds__(kEwThreads, 4)
 k_scale_cols_strip_bf16(const MatTable t, double* partials) {
@@ -1164,10 +1092,9 @@ cudaError_t launch_epilogue_flat(const MatTable& t, int nblk, float lr, int upda
   k_epilogue_flat<<<nblk, kEwThreads, 0, st>>>(t, lr, update_w, scal);
   return cudaGetLastError();
 }
-cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, float beta,
-                           cudaStream_t st) {
+cudaError_t launch_colnorm(const MatTable& t, int nblk, float pp_eps, float beta, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
-  k_colnorm<<<nblk, kEwThreads, 0, st>>>(t, mode, pp_eps, beta);
+  k_colnorm<<<nblk, kEwThreads, 0, st>>>(t, pp_eps, beta);
   return cudaGetLastError();
 }
 cudaError_t launch_colsq_partial(const MatTable& t, int nblk, cudaStream_t st) {
@@ -1222,11 +1149,6 @@ cudaError_t launch_prologue_tall_bf16(const MatTable& t, int nblk, float mu, int
 cudaError_t launch_scale_cols_strip_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
   if (nblk == 0) return cudaSuccess;
   k_scale_cols_strip_bf16<<<nblk, kEwThreads, 0, st>>>(t, partials);
-  return cudaGetLastError();
-}
-cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st) {
-  if (nblk == 0) return cudaSuccess;
-  k_scale_cols_flat_bf16<<<nblk, kEwThreads, 0, st>>>(t, partials);
   return cudaGetLastError();
 }
 cudaError_t launch_epilogue_flat_bf16(const MatTable& t, int nblk, float lr, int update_w, const double* scal,

@@ -722,7 +722,7 @@ muon_status stage_polar(const Ctx& c, bool aurora) {
       }));
       CK(for_chunks(c, fq.second, [](const MatDesc& d) { return cdiv(d.l, kColStrip); }, [&](const MatTable& t, int nb) {
         ProfScope ps(PC_AURORA, 0.0, c.plan->nsb * table_elems(t), c.st);
-        return launch_colnorm(t, nb, 1, pe, beta, c.st);
+        return launch_colnorm(t, nb, pe, beta, c.st);
       }));
     }
   }

@@ -86,8 +86,8 @@ cudaError_t launch_prologue(const MatTable& t, int nblk, int mode, float mu, int
                             int want_w2, double* partials, cudaStream_t st);
 cudaError_t launch_finalize_sums(const MatTable& t, const double* partials, int nq, int slot0,
                                  int slot1, double* scal, cudaStream_t st);
-cudaError_t launch_colnorm(const MatTable& t, int nblk, int mode, float pp_eps, float beta,
-                           cudaStream_t st);
+// Aurora D update from a pass over U (FP32 / SIMT modes).
+cudaError_t launch_colnorm(const MatTable& t, int nblk, float pp_eps, float beta, cudaStream_t st);
 cudaError_t launch_scale_cols(const MatTable& t, int nblk, double* partials, cudaStream_t st);
 // Aurora D from per-row-block column sums of squares (MatDesc::colsq):
 // k_colsq_partial forms them from uX per kColsqRows rows (blocks of
@@ -109,9 +109,8 @@ cudaError_t launch_epilogue(const MatTable& t, int nblk, float lr, int update_w,
 // Optimizer-step prologue, tall, m and n multiples of 64, bf16 grads / params / NS storage.
 cudaError_t launch_prologue_tall_bf16(const MatTable& t, int nblk, float mu, int nesterov, int want_w2,
                                       double* partials, cudaStream_t st);
-// Flat Aurora input scaling with bf16 NS storage.
-cudaError_t launch_scale_cols_flat_bf16(const MatTable& t, int nblk, double* partials, cudaStream_t st);
-// The same by column strips: blocks of kStripCols columns x kStripRows rows,
+// Aurora input scaling with bf16 NS storage and contiguous rows, by column
+// strips: blocks of kStripCols columns x kStripRows rows,
 // one partial slot per block (cdiv(l, kStripCols) * cdiv(s, kStripRows) of
 // them, never more than the matrix's 64 x 64 tiles).
 constexpr int kStripCols = 2048, kStripRows = 64;
