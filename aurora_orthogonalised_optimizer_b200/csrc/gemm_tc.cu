@@ -23,7 +23,8 @@
 // alpha*acc + beta*E, a 32 x 32 bf16 block staged in shared memory with the
 // 64-byte swizzle, TMA bulk-tensor store.  A and A^2 are symmetric: only tiles
 // touching the upper triangle run; each stores its upper blocks directly and
-// mirrored, and the diagonal block is completed from its own upper triangle,
+// mirrored (the transposed block built from 8 x 8 tiles with ldmatrix.trans /
+// stmatrix), and the diagonal block is completed from its own upper triangle,
 // so every element is written exactly once.
 // Operand majorness: Gram and square read both operands K-major; the update
 // reads X as an MN-major B operand (X is [K][N] with N contiguous).
@@ -145,23 +146,45 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
-__device__ __forceinline__ void st_shared_u16(uint32_t a, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
-}
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
   return v;
 }
-__device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
-  return v;
+__device__ __forceinline__ void ld_shared_v4(uint32_t a, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(a) : "memory");
 }
 // Byte offset of (row r, byte b) inside a 32 x 64-byte block stored with the
 // TMA 64-byte swizzle: 16-byte chunk index XOR ((r >> 1) & 3).
 __device__ __forceinline__ uint32_t swz64(int r, int b) {
   return (uint32_t)(r * 64 + ((((b >> 4) ^ (r >> 1)) & 3) << 4) + (b & 15));
+}
+// Four 8 x 8 tiles of 16-bit values between shared memory and registers; in
+// registers lane t holds row t / 4, columns 2 (t % 4) and 2 (t % 4) + 1 of
+// tile i in x_i, and lanes 8i .. 8i + 7 give the addresses of tile i's rows.
+// The load transposes each tile.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t a, uint32_t& x0, uint32_t& x1, uint32_t& x2, uint32_t& x3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+               : "r"(a)
+               : "memory");
+}
+__device__ __forceinline__ void stsm_x4(uint32_t a, uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x0), "r"(x1), "r"(x2),
+               "r"(x3)
+               : "memory");
+}
+// dst <- the transpose of the 32 x 32 block of 16-bit values at src (both
+// 64-byte swizzled).  Step a moves tiles (a, 0..3) of src to tiles (0..3, a)
+// of dst, each transposed on the way through registers.
+__device__ __forceinline__ void transpose_block32(uint32_t src, uint32_t dst, int lane) {
+  const int m = lane >> 3, rr = lane & 7;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    uint32_t x0, x1, x2, x3;
+    ldsm_x4_trans(src + swz64(8 * a + rr, 16 * m), x0, x1, x2, x3);
+    stsm_x4(dst + swz64(8 * m + rr, 16 * a), x0, x1, x2, x3);
+  }
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
@@ -587,18 +610,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           st_shared_v4(dbuf + swz64(lane, 16 * c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         const bool diag = sym && col0 == r0;
         const bool mirror = sym && col0 > r0;
+        if (diag || mirror) {
+          // the transposed block: the mirror's store, or (diagonal block)
+          // the source of its lower part
+          __syncwarp();
+          transpose_block32(dbuf, mbuf, lane);
+        }
         if (diag) {
           __syncwarp();
-          // lower part of the diagonal block <- its upper part (element (j, lane) of row j)
-          for (int j = 0; j < lane; ++j) {
-            const uint16_t h = ld_shared_u16(dbuf + swz64(j, 2 * lane));
-            st_shared_u16(dbuf + swz64(lane, 2 * j), h);
-          }
-        }
-        if (mirror) {
+          // lower part of the diagonal block <- its upper part: row `lane`
+          // takes the columns left of the diagonal from the transposed copy
+          uint32_t tw[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            st_shared_u16(mbuf + swz64(j, 2 * lane), (uint16_t)(pk[j >> 1] >> (16 * (j & 1))));
+          for (int c = 0; c < 4; ++c) ld_shared_v4(mbuf + swz64(lane, 16 * c), tw[4 * c], tw[4 * c + 1], tw[4 * c + 2], tw[4 * c + 3]);
+#pragma unroll
+          for (int w = 0; w < 16; ++w) {
+            if (2 * w + 1 < lane) pk[w] = tw[w];
+            else if (2 * w < lane) pk[w] = (pk[w] & 0xFFFF0000u) | (tw[w] & 0xFFFFu);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_shared_v4(dbuf + swz64(lane, 16 * c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
         if (G.colsq) {
           // column sums of the squared stored values of this 32 x 32 block:
