@@ -535,9 +535,7 @@ void add_group(const Ctx& c, GemmLaunch& L, GemmGroup g) {
   if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
     g.tiles_per_mat = tc_tile_count(g.kind, g.M, g.N, tc_pair(), &g.tiles_m, &g.tiles_n);
   } else {
-    g.tiles_m = (int)cdiv(g.M, 64);
-    g.tiles_n = (int)cdiv(g.N, 64);
-    g.tiles_per_mat = g.tiles_m * g.tiles_n;
+    g.tiles_per_mat = simt_tile_count(g.kind, g.M, g.N, &g.tiles_m, &g.tiles_n);
   }
   g.tile_begin = L.total_tiles;
   L.g[L.num_groups++] = g;

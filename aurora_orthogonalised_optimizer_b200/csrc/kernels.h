@@ -54,7 +54,11 @@ struct GemmLaunch {
   GemmGroup g[kMaxGemmGroups];
 };
 
-// SIMT grouped GEMM (fp32 FMA accumulation; bf16 or fp32 storage).
+// SIMT grouped GEMM (fp32 FMA accumulation; bf16 or fp32 storage): tiles of
+// kSimtTile x kSimtTile outputs; the symmetric kinds run only the tiles on or
+// above the diagonal (simt_tile_count gives a group's tiles per matrix).
+constexpr int kSimtTile = 128;
+int simt_tile_count(int kind, int M, int N, int* tiles_m, int* tiles_n);
 cudaError_t launch_gemm_simt(const GemmLaunch& L, cudaStream_t st);
 
 // tcgen05 grouped GEMM (bf16 operands, fp32 accumulation in TMEM, TMA loads).
