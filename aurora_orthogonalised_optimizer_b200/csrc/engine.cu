@@ -56,7 +56,7 @@ struct Plan {
   int nsb = 2;
   std::vector<MatPlan> mats;
   std::vector<BucketPlan> buckets;
-  size_t off_scal = 0, off_partials = 0, off_gv = 0, off_dots = 0, total = 0;
+  size_t off_scal = 0, off_partials = 0, off_gv = 0, off_dots = 0, off_sched = 0, total = 0;
 };
 
 // Rows per item of the fused power-iteration pass: items of about
@@ -149,6 +149,8 @@ Plan make_plan(const muon_config* cfg, int n, const muon_shape* shapes) {
   off = align_up(off + (size_t)part * 8 /*warps*/ * 2 * sizeof(double));
   p.off_gv = off;
   off = align_up(off + (size_t)gv * sizeof(float));
+  p.off_sched = off;                                   // the tensor-core GEMM's tile counter
+  off = align_up(off + sizeof(unsigned int));
   p.total = off;
   return p;
 }
@@ -281,6 +283,7 @@ struct Ctx {
   cudaStream_t st;
   double* scal;
   double* partials;
+  unsigned int* sched;    // tile counter of the tensor-core GEMM launches
   void* const* W;
   const void* const* G;
   float* const* M;
@@ -519,6 +522,8 @@ muon_status gemm_launch(const Ctx& c, GemmLaunch& L) {
   if (c.cfg->gemm_mode == MUON_GEMM_BF16) {
     alignas(64) unsigned char maps[kMaxGemmGroups * 3 * 128];
     if (!tc_encode_maps(L, tc_pair(), maps)) return MUON_ERR_CUDA;
+    L.tile_ctr = c.sched;
+    CK(cudaMemsetAsync(c.sched, 0, sizeof(unsigned int), c.st));
     ProfScope ps(PC_GEMM_TC, gemm_flops(L), 0.0, c.st);
     ProfScope pk(PC_TC_GRAM + L.g[0].kind, gemm_flops(L), 0.0, c.st);   // every group of a launch has one kind
     CK(launch_gemm_tc(L, maps, num_sms_current(), tc_pair(), c.st));
@@ -812,6 +817,7 @@ Ctx make_ctx(const muon_config* cfg, const Plan& p, void* ws, void* stream) {
   c.st = reinterpret_cast<cudaStream_t>(stream);
   c.scal = reinterpret_cast<double*>(c.ws + p.off_scal);
   c.partials = reinterpret_cast<double*>(c.ws + p.off_partials);
+  c.sched = reinterpret_cast<unsigned int*>(c.ws + p.off_sched);
   c.param_dtype = cfg->param_dtype;
   c.grad_dtype = cfg->grad_dtype;
   return c;

@@ -16,6 +16,12 @@
 //     both CTAs complete on the leader's barrier) and owns 128 rows of the
 //     fp32 accumulator in its TMEM.  6-stage ring of 2 x 16 KiB per CTA.
 //     Per FLOP this halves the B traffic of each SM.
+// Tiles are taken in launch order from a device counter (L.tile_ctr) as each
+// CTA (pair) frees up, so the tiles in flight at any moment are neighbours
+// in that order and their operands stay in L2; with a fixed round-robin
+// deal, the units drift apart over hundreds of waves and the operands of
+// several matrices compete for L2 (about 3x the operand bytes read from
+// DRAM on the 168-matrix step).
 // Roles: warp 0 = TMA producer (one lane); warp 1 = TMEM allocator and MMA
 // issuer (one lane of the leader); warps 2..5 = epilogue.  Two 256-column
 // TMEM accumulators let the epilogue of one tile overlap the main loop of the
@@ -57,6 +63,12 @@ constexpr uint32_t kTmemCols = 512;                   // 2 accumulators x 256 fp
 constexpr uint32_t kOutTileBytes = 32 * 32 * 2;       // one staged 32x32 bf16 output block
 constexpr uint32_t kOutBytes = 4 /*warps*/ * 4 /*2 parities x {direct, mirror}*/ * kOutTileBytes;
 constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
+constexpr int kTq = 4;                                // slots of the tile-index ring
+// threads that free each ring slot: the MMA issuer and the four epilogue
+// warps of the leader CTA, and (SM pair) the producer and the four epilogue
+// warps of the peer
+template <bool PAIR>
+constexpr uint32_t kTqTakers = PAIR ? 10u : 5u;
 
 // Per-variant geometry (see the file comment).
 template <bool PAIR>
@@ -68,7 +80,7 @@ struct Geo {
   static constexpr uint32_t kBBytes = kBRows * TBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * kStageBytes;    // lands on the leader's barrier
-  static constexpr size_t kSmemBytes = 1024 + kStages * (size_t)kStageBytes + kOutBytes + 256;
+  static constexpr size_t kSmemBytes = 1024 + kStages * (size_t)kStageBytes + kOutBytes + 512;
 };
 static_assert(Geo<true>::kSmemBytes <= 232448 && Geo<false>::kSmemBytes <= 232448, "shared memory budget");
 
@@ -101,14 +113,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same with acquire at cluster scope: the phase was completed by a
+// release from another CTA of the cluster whose shared-memory writes the
+// waiter then reads.
+__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait; returns false (and raises the abort flag) on timeout or when
-// another role already aborted.
+// another role already aborted.  `cl`: acquire at cluster scope.
 __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag,
-                                          long long limit = kWaitLimitCycles) {
-  if (mbar_try_wait(a, parity)) return true;
+                                          long long limit = kWaitLimitCycles, bool cl = false) {
+  auto try_once = [&]() { return cl ? mbar_try_wait_cl(a, parity) : mbar_try_wait(a, parity); };
+  if (try_once()) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (try_once()) return true;
     if ((i & 255u) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) {
@@ -218,16 +245,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-__device__ __forceinline__ uint32_t cluster_id() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_count() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-  return r;
-}
 // shared::cluster address of the same shared-memory offset in CTA `rank`
 __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
   uint32_t r;
@@ -236,6 +253,14 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
 }
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+// Arrive on a peer CTA's barrier, ordering this thread's earlier shared-memory
+// writes to the peer (st.shared::cluster) before it at cluster scope.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t a) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t a) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
@@ -379,13 +404,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   const uint32_t tfull0 = empty0 + 8 * S, tempty0 = tfull0 + 16, drain = tempty0 + 16;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(ctl + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 196);
+  // ring of tile indices: full[kTq], empty[kTq], index[kTq]
+  const uint32_t tqf0 = smem_u32(ctl + 256), tqe0 = tqf0 + 8 * kTq;
+  const uint32_t tq_addr = tqe0 + 8 * kTq;
+  volatile int* tq = reinterpret_cast<volatile int*>(ctl + 256 + 16 * kTq);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GemmLaunch& L = P.L;
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const bool leader = rank == 0;
-  const int unit = PAIR ? (int)cluster_id() : (int)blockIdx.x;      // tile-processing unit
-  const int units = PAIR ? (int)cluster_count() : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -397,6 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       mbar_init(tempty0 + 8 * a, (PAIR ? 2 : 1) * 4);   // one arrive per epilogue warp of each CTA
     }
     mbar_init(drain, 1);
+    for (int k = 0; k < kTq; ++k) {
+      mbar_init(tqf0 + 8 * k, 1);
+      mbar_init(tqe0 + 8 * k, kTqTakers<PAIR>);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -413,6 +444,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // The tile sequence.  The leader CTA's producer takes each next tile index
+  // from L.tile_ctr as it starts a tile and publishes it in its ring slot
+  // (and, SM pair, in the peer CTA's); the MMA issuer, the epilogue warps and
+  // the peer's producer read the slots in order and free each on the
+  // leader's barrier.  -1 ends the sequence; -2 means a wait gave up.
+  auto tq_advance = [&](int& qi, uint32_t& qph) {
+    if (++qi == kTq) { qi = 0; qph ^= 1u; }
+  };
+  auto tq_publish = [&](int& qi, uint32_t& qph) -> int {
+    if (!mbar_wait(tqe0 + 8 * qi, qph ^ 1u, abort_flag)) return -2;
+    int t = (int)atomicAdd(L.tile_ctr, 1u);
+    if (t >= L.total_tiles) t = -1;
+    tq[qi] = t;
+    if constexpr (PAIR) {
+      st_cluster_u32(map_to_rank(tq_addr + 4 * qi, 1), (uint32_t)t);
+      mbar_arrive_release_cluster(map_to_rank(tqf0 + 8 * qi, 1));
+    }
+    mbar_arrive(tqf0 + 8 * qi);
+    tq_advance(qi, qph);
+    return t;
+  };
+  auto tq_read = [&](int qi, uint32_t qph) -> int {
+    if (!mbar_wait(tqf0 + 8 * qi, qph, abort_flag, kWaitLimitCycles, PAIR)) return -2;
+    return tq[qi];
+  };
+  auto tq_free = [&](int qi) {   // after the slot's index has been read
+    if constexpr (PAIR) {
+      if (leader) mbar_arrive(tqe0 + 8 * qi);
+      else mbar_arrive_release_cluster(map_to_rank(tqe0 + 8 * qi, 0));
+    } else {
+      mbar_arrive(tqe0 + 8 * qi);
+    }
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -420,7 +485,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
-      for (int tile = unit; tile < L.total_tiles && ok; tile += units) {
+      int qi = 0;
+      uint32_t qph = 0;
+      for (;;) {
+        int tile;
+        if (leader) {
+          tile = tq_publish(qi, qph);
+        } else {
+          tile = tq_read(qi, qph);
+          if (tile != -2) tq_free(qi);
+          tq_advance(qi, qph);
+        }
+        if (tile == -2) { ok = false; break; }
+        if (tile < 0) break;
         const TileInfo ti = decode_tile<PAIR>(L, tile);
         const GemmGroup& G = L.g[ti.g];
         const CUtensorMap* mA = &P.maps[3 * ti.g];
@@ -456,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           ++issued;
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
+        if (!ok) break;
       }
       if (!ok && leader) {
         // drain: wait (bounded) for every stage's most recent loads (of both
@@ -475,7 +553,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, any = false;
       int it = 0;
-      for (int tile = unit; tile < L.total_tiles && ok; tile += units, ++it) {
+      int qi = 0;
+      uint32_t qph = 0;
+      for (;; ++it) {
+        const int tile = tq_read(qi, qph);
+        if (tile == -2) { ok = false; break; }
+        tq_free(qi);
+        tq_advance(qi, qph);
+        if (tile < 0) break;
         const TileInfo ti = decode_tile<PAIR>(L, tile);
         const bool upd = L.g[ti.g].kind == GK_UPD;
         const uint32_t idesc = make_idesc(upd ? 1u : 0u, (uint32_t)Gm::kTileM);
@@ -522,7 +607,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     const uint32_t tempty_leader0 = PAIR ? map_to_rank(tempty0, 0) : tempty0;
     uint32_t acc_phase = 0, par = 0;
     int it = 0;
-    for (int tile = unit; tile < L.total_tiles; tile += units, ++it) {
+    int qi = 0;
+    uint32_t qph = 0;
+    for (;; ++it) {
+      // lane 0 takes the next index for the warp
+      int tile = 0;
+      if (lane == 0) {
+        tile = tq_read(qi, qph);
+        if (tile != -2) tq_free(qi);
+      }
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      tq_advance(qi, qph);
+      if (tile < 0) break;
       const TileInfo ti = decode_tile<PAIR>(L, tile);
       const GemmGroup& G = L.g[ti.g];
       const int acc = it & 1;

@@ -51,6 +51,9 @@ struct GemmLaunch {
   int num_groups;
   int total_tiles;
   int dtype;                      // kF32 or kBF16
+  // tensor-core path: the next tile to take (device counter, zero at launch);
+  // each CTA (pair) takes tiles in this order as it frees up
+  unsigned int* tile_ctr;
   GemmGroup g[kMaxGemmGroups];
 };
 
