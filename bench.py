@@ -559,7 +559,7 @@ def main():
     if args.graph:
         if world > 1:
             raise SystemExit("--graph is for one GPU")
-        # the step issues only kernel launches on its stream: capture one and replay it
+        # the step issues only kernel launches and workspace memsets on its stream: capture one and replay it
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             A.muon_step(cfg, params, grads, mom, None, ws)

@@ -108,10 +108,11 @@ size_t muon_workspace_size(const muon_config* cfg, int n, const muon_shape* shap
  * momentum : n device pointers, fp32, updated in place.
  * update_out: NULL, or n device pointers (entries may be NULL) receiving V
  *            in fp32 (m x n), the applied update before the lr.
- * The call only enqueues kernel launches on `stream` (no allocation, no
- * synchronisation, no host read of device data), so it can be captured in a
- * CUDA graph once the first call on the device has been made outside
- * capture; the captured launches carry this call's config.
+ * The call only enqueues kernel launches, and 4-byte memsets of the
+ * workspace (the tensor-core GEMM's tile counter), on `stream` (no
+ * allocation, no synchronisation, no host read of device data), so it can be
+ * captured in a CUDA graph once the first call on the device has been made
+ * outside capture; the captured launches carry this call's config.
  * Errors: INVALID_ARG, WORKSPACE, CUDA as described above. */
 muon_status muon_step(const muon_config* cfg, int n, const muon_shape* shapes,
                       void* const* params, const void* const* grads,

@@ -1,6 +1,7 @@
 """muon_step inside a CUDA graph: the entry point issues only kernel launches
-on the caller's stream (no allocation, no synchronisation, no host read of
-device data), so a captured step replays to the same bits as an eager one.
+and workspace memsets on the caller's stream (no allocation, no
+synchronisation, no host read of device data), so a captured step replays to
+the same bits as an eager one.
 This is what lets a launch-bound caller (small matrices, ~125 launches per
 step) replace the per-launch host cost with one graph launch."""
 import pytest
