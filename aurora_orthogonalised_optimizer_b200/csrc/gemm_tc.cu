@@ -453,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     if (++qi == kTq) { qi = 0; qph ^= 1u; }
   };
   auto tq_publish = [&](int& qi, uint32_t& qph) -> int {
-    if (!mbar_wait(tqe0 + 8 * qi, qph ^ 1u, abort_flag)) return -2;
+    // (the peer's frees are released at cluster scope: acquire at cluster scope)
+    if (!mbar_wait(tqe0 + 8 * qi, qph ^ 1u, abort_flag, kWaitLimitCycles, PAIR)) return -2;
     int t = (int)atomicAdd(L.tile_ctr, 1u);
     if (t >= L.total_tiles) t = -1;
     tq[qi] = t;
